@@ -1,0 +1,433 @@
+"""Benchmark of the SambaY scan + Gated Memory Unit hot path on B200.
+
+One step = one pass of the prefill hot path over one batch: the Mamba
+selective scan of a 2048-token prompt (batch 1, d_inner 5120, d_state 16,
+conv 4, dt_rank 160) writing the memory readout M, then one GMU layer
+Y = (M ⊙ SiLU(X W1^T)) W2 with d_model 2560, in bfloat16 I/O with float32
+accumulation and state.  Metric: tokens/s over the step.  A decode
+sub-benchmark (64 sequences, one token each per step: scan step + GMU step)
+is reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU, each an independent replica
+(weak scaling: the sequences of different ranks share nothing, so there is
+no collective on the data path).  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_memory_sharing_b200 import synth  # noqa: E402
+
+WORKLOAD = "prefill_b1_l2048"
+METRIC = "scan+GMU prefill tokens/s"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
+DECODE_BATCH = 64
+DECODE_RING = 64             # decode steps per captured graph
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        # median over the samples taken under load (top half of power draw)
+        if power:
+            cut = statistics.median(power)
+            loaded = [s for s, p in zip(sm, power) if p >= cut] or sm
+        else:
+            loaded = sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    """The float64 oracle on the host cores, on a bounded sample per step."""
+    if rank != 0:
+        return
+    from oracle import sambay_ref as ref
+    d, seed = synth.workload(WORKLOAD)
+    w = synth.scan_weights(d, seed)
+    gw = synth.gmu_weights(d, seed)
+    sample = 256
+    u = synth.scan_inputs(d, seed, seqlen=sample)
+    X = synth.gmu_inputs(d, seed, rows=sample)
+
+    def step():
+        r = ref.scan_prefill_ref(u, w)
+        ref.gmu_ref(X, r["M"][0], gw["W1"], gw["W2"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * sample / el
+    cores = len(os.sched_getaffinity(0))
+    desc = f"first {sample} tokens of the {d.seqlen}-token prompt (scan + GMU rows) per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": d.batch, "seq_len": d.seqlen,
+                   "d_model": d.d_model, "d_inner": d.d_inner, "d_state": d.d_state,
+                   "sample_tokens": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def cpu_baseline_oracle(min_seconds=10.0, max_reps=4):
+    """The oracle as it stands, on the full benchmark step, timed on this host."""
+    from oracle import sambay_ref as ref
+    d, seed = synth.workload(WORKLOAD)
+    w = synth.scan_weights(d, seed)
+    gw = synth.gmu_weights(d, seed)
+    u = synth.scan_inputs(d, seed)
+    X = synth.gmu_inputs(d, seed)
+    reps, t0 = 0, time.perf_counter()
+    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_seconds):
+        r = ref.scan_prefill_ref(u, w)
+        ref.gmu_ref(X, r["M"][0], gw["W1"], gw["W2"])
+        reps += 1
+    el = time.perf_counter() - t0
+    return {"value": reps * d.tokens / el, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"the whole step ({d.tokens} tokens: scan + one GMU layer) x {reps}, "
+                      f"{el:.1f} s of float64 NumPy"}
+
+
+# --------------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    from gated_memory_sharing_b200 import abi, build
+    from gated_memory_sharing_b200.layers import GMULayer, ScanLayer, to_device
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    if rank == 0:
+        build.build()
+    barrier(world)
+    abi.load()
+    peaks, peak_kind = load_peaks()
+
+    d, seed = synth.workload(WORKLOAD)
+    w = synth.scan_weights(d, seed)
+    gw = synth.gmu_weights(d, seed)
+    # each rank: its own sequence (weak scaling), the same weights
+    u_np = synth.scan_inputs(d, seed + 7919 * rank)
+    X_np = synth.gmu_inputs(d, seed + 7919 * rank)
+    scan = ScanLayer(w, d.d_model, abi.BF16)
+    gmu = GMULayer(gw["W1"], gw["W2"], abi.BF16)
+    u = to_device(u_np, abi.BF16)
+    X = to_device(X_np, abi.BF16)
+    T, Di, Dm = d.tokens, d.d_inner, d.d_model
+    M = torch.empty_like(u)
+    Y = torch.empty_like(X)
+    h, cs = scan.new_state(d.batch)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        scan.prefill(u, h, cs, M=M, fresh=True)
+
+    def gmu_step():
+        gmu.forward(X, M.view(T, Di), residual=False, Y=Y)
+
+    # warm-up (also sets kernel attributes outside the timed region)
+    for _ in range(max(args.warmup, 3)):
+        step()
+        gmu_step()
+    torch.cuda.synchronize()
+    assert abi.sambay_device_status() == 0
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+
+    # ---- device-resident timed region: K steps, L2 flushed between steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+        gmu_step()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    scan_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    gmu_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    step_ms = [a + b for a, b in zip(scan_ms, gmu_ms)]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    value = world * args.steps * T / (total_ms / 1e3)
+    launches_per_step = 5 + 2   # conv, x_proj GEMM, x_proj reduce, dt_proj GEMM, scan; 2 GMU GEMMs
+
+    # ---- end to end through the ABI with host buffers
+    u_host = u.cpu().pin_memory()
+    X_host = X.cpu().pin_memory()
+    Y_host = torch.empty(Y.shape, dtype=Y.dtype).pin_memory()
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        ev2[i][0].record(stream)
+        u.copy_(u_host, non_blocking=True)
+        X.copy_(X_host, non_blocking=True)
+        step()
+        gmu_step()
+        Y_host.copy_(Y, non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(args.steps)),
+                            world, device)
+    e2e_value = world * args.steps * T / (e2e_ms / 1e3)
+
+    # ---- decode sub-benchmark: 64 sequences, one token each per step
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(args, scan, gmu, d, seed + 7919 * rank, flush, stream, world, device, peaks)
+    clk = clocks.stop()
+    assert abi.sambay_device_status() == 0
+
+    # ---- roofline of the dominant kernel pair (the GMU's two tcgen05 GEMMs)
+    gmu_mean_ms = statistics.mean(gmu_ms)
+    gmu_flops = 4.0 * T * Dm * Di
+    achieved_tf = gmu_flops / (gmu_mean_ms / 1e3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": None,
+                "kernel": "gmu_forward: tc_gemm_kernel x2 (X W1^T + gate, H W2)",
+                "peak_kind": f"{peak_kind} burst bf16"}
+    scan_mean_ms = statistics.mean(scan_ms)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": d.batch, "seq_len": d.seqlen,
+                   "d_model": Dm, "d_inner": Di, "d_state": d.d_state, "d_conv": d.d_conv,
+                   "dt_rank": d.dt_rank, "gmu_layers": 1, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between steps (256 MB write, outside the step events)"},
+        "roofline": roofline,
+        "breakdown_ms": {"scan_prefill": scan_mean_ms, "gmu_forward": gmu_mean_ms},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": u.numel() * 2 + X.numel() * 2,
+                "d2h_bytes_per_step": Y.numel() * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if decode is not None:
+        out["decode"] = decode
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_oracle()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    barrier(world)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def bench_decode(args, scan, gmu, d, seed, flush, stream, world, device, peaks):
+    import torch
+    from gated_memory_sharing_b200.layers import to_device
+    B, Di, Dm = DECODE_BATCH, d.d_inner, d.d_model
+    dd = synth.Dims(B, 16, Dm, Di, d.d_state, d.d_conv, d.dt_rank, synth.BF16)
+    u0 = to_device(synth.scan_inputs(dd, seed + 1), 1)                       # 16-token prompt
+    ring_u = to_device(synth.scan_inputs(dd, seed + 2, seqlen=DECODE_RING, tag="u_dec"), 1)
+    ring_x = to_device(synth.gmu_inputs(dd, seed + 3, rows=B * DECODE_RING, tag="X_dec"), 1)
+    ring_u = ring_u.transpose(0, 1).contiguous()                              # [ring, B, Di]
+    ring_x = ring_x.view(DECODE_RING, B, Dm)
+    _, h, cs = scan.prefill(u0)
+    m = torch.empty(B, Di, dtype=torch.bfloat16, device=device)
+    y = torch.empty(DECODE_RING, B, Dm, dtype=torch.bfloat16, device=device)
+
+    def steps():
+        for i in range(DECODE_RING):
+            scan.step(ring_u[i], h, cs, m_t=m)
+            gmu.step(ring_x[i], m, residual=True, Y=y[i])
+
+    steps()                      # warm-up, workspaces, kernel attributes
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        steps()
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(args.steps // 4, 5)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(reps):
+        flush.fill_(float(i))
+        ev[i][0].record(stream)
+        g.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    step_us = 1e3 * total_ms / (reps * DECODE_RING)
+    # algorithmic bytes per decode step (every byte the step must move once)
+    state = B * Di * d.d_state * 4 * 2 + B * Di * d.d_conv * 2 * 2
+    weights = (d.dt_rank + 2 * d.d_state) * Di * 2 + Di * d.dt_rank * 2 + Di * (d.d_conv + 1) * 2 \
+        + Di * d.d_state * 4 + 2 * Di * 4 + 2 * Di * Dm * 2
+    acts = B * (2 * Di + 3 * Dm) * 2
+    nbytes = state + weights + acts
+    achieved = nbytes / (step_us / 1e6) / 1e9
+    del g
+    return {"metric": "decode tokens/s (scan step + GMU step)", "unit": UNIT,
+            "value": world * B / (step_us / 1e6), "us_per_step": step_us, "batch": B,
+            "steps_timed": reps * DECODE_RING,
+            "setup": "16-token prompt prefill; the decode state has a fixed size, so the step "
+                     "cost does not depend on the position",
+            "l2": "flushed between graph replays of 64 back-to-back steps",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_step": nbytes}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

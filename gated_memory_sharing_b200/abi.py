@@ -1,0 +1,199 @@
+"""Thin ctypes binding of libsambay (the C ABI in ``include/sambay.h``).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the current CUDA device, passes their ``data_ptr()`` and the current
+CUDA stream to the C entry point of the same name, and raises
+:class:`SambayError` on a non-OK status.  There is no fallback: if the
+library has not been built, importing the symbols raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "lib", "libsambay.so")
+
+F32 = 0
+BF16 = 1
+
+STATUS = {
+    0: "SAMBAY_OK",
+    1: "SAMBAY_ERR_INVALID_ARG",
+    2: "SAMBAY_ERR_UNSUPPORTED",
+    3: "SAMBAY_ERR_WORKSPACE",
+    4: "SAMBAY_ERR_CUDA",
+    5: "SAMBAY_ERR_TIMEOUT",
+    6: "SAMBAY_ERR_DEVICE",
+}
+
+EXPORTS = (
+    "sambay_scan_prefill_workspace",
+    "sambay_scan_step_workspace",
+    "gmu_forward_workspace",
+    "gmu_step_workspace",
+    "sambay_scan_prefill",
+    "sambay_scan_step",
+    "gmu_forward",
+    "gmu_step",
+    "sambay_device_status",
+    "sambay_status_string",
+    "sambay_version",
+)
+
+
+class SambayError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("seqlen", ctypes.c_int32),
+        ("d_model", ctypes.c_int32),
+        ("d_inner", ctypes.c_int32),
+        ("d_state", ctypes.c_int32),
+        ("d_conv", ctypes.c_int32),
+        ("dt_rank", ctypes.c_int32),
+        ("io", ctypes.c_int32),
+    ]
+
+
+class ScanWeights(ctypes.Structure):
+    _fields_ = [
+        ("conv_w", ctypes.c_void_p),
+        ("conv_b", ctypes.c_void_p),
+        ("x_proj_w", ctypes.c_void_p),
+        ("dt_proj_w", ctypes.c_void_p),
+        ("dt_bias", ctypes.c_void_p),
+        ("A", ctypes.c_void_p),
+        ("D", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsambay once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libsambay is not built ({path} missing): run "
+            "`python -m gated_memory_sharing_b200.build` or __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
+    pd, pw = ctypes.POINTER(Dims), ctypes.POINTER(ScanWeights)
+    sig = {
+        "sambay_scan_prefill_workspace": (sz, [pd]),
+        "sambay_scan_step_workspace": (sz, [pd]),
+        "gmu_forward_workspace": (sz, [pd, i64]),
+        "gmu_step_workspace": (sz, [pd, i64]),
+        "sambay_scan_prefill": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]),
+        "sambay_scan_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp, sz, vp]),
+        "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sambay_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
+        "sambay_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "sambay_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------------- marshalling
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL)."""
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise SambayError(fn, code)
+
+
+def make_dims(batch, seqlen, d_model, d_inner, d_state=16, d_conv=4, dt_rank=160, io=BF16) -> Dims:
+    return Dims(batch, seqlen, d_model, d_inner, d_state, d_conv, dt_rank, io)
+
+
+def make_weights(conv_w, conv_b, x_proj_w, dt_proj_w, dt_bias, A, D) -> ScanWeights:
+    return ScanWeights(*(t.data_ptr() for t in (conv_w, conv_b, x_proj_w, dt_proj_w, dt_bias, A, D)))
+
+
+def sambay_scan_prefill_workspace(dims: Dims) -> int:
+    return load().sambay_scan_prefill_workspace(ctypes.byref(dims))
+
+
+def sambay_scan_step_workspace(dims: Dims) -> int:
+    return load().sambay_scan_step_workspace(ctypes.byref(dims))
+
+
+def gmu_forward_workspace(dims: Dims, rows: int) -> int:
+    return load().gmu_forward_workspace(ctypes.byref(dims), rows)
+
+
+def gmu_step_workspace(dims: Dims, rows: int) -> int:
+    return load().gmu_step_workspace(ctypes.byref(dims), rows)
+
+
+def sambay_scan_prefill(weights: ScanWeights, dims: Dims, u, M, ssm_state, conv_state,
+                        zero_init_state: bool, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_scan_prefill", load().sambay_scan_prefill(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u), _p(M), _p(ssm_state), _p(conv_state),
+        1 if zero_init_state else 0, _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_scan_step(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv_state, ws,
+                     stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_scan_step", load().sambay_scan_step(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state),
+        _p(conv_state), _p(ws), ws_bytes, _stream(stream)))
+
+
+def gmu_forward(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("gmu_forward", load().gmu_forward(
+        ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(residual), _p(Y), _p(ws),
+        ws_bytes, _stream(stream)))
+
+
+def gmu_step(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("gmu_step", load().gmu_step(
+        ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(residual), _p(Y), _p(ws),
+        ws_bytes, _stream(stream)))
+
+
+def sambay_device_status(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check("sambay_device_status", load().sambay_device_status(_stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+def sambay_status_string(code: int) -> str:
+    return load().sambay_status_string(code).decode()
+
+
+def sambay_version() -> str:
+    return load().sambay_version().decode()

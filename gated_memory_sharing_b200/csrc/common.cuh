@@ -1,0 +1,58 @@
+// Shared device helpers for the SambaY scan + GMU kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sambay {
+
+// Per-device status word.  A kernel that detects a fault (a bounded wait that
+// ran out) records the first code here; sambay_device_status reads and
+// clears it.  Module-scope storage, not an allocation.
+__device__ int g_status;
+
+__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
+
+constexpr int kStatusTimeout = 5;  // == SAMBAY_ERR_TIMEOUT
+
+typedef __nv_bfloat16 bf16;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// SiLU(x) = x / (1 + e^-x), the GMU gate activation and Mamba's post-conv one.
+__device__ __forceinline__ float silu(float x) {
+  return __fdividef(x, 1.0f + ex2_approx(-x * kLog2e));
+}
+
+// softplus(x) = log(1 + e^x).  Above 20 the correction log1p(e^-x) < 2.1e-9
+// relative, below float32 resolution of x, so x is returned there; otherwise
+// log1p of the exponential, with CUDA's own log1pf.
+__device__ __forceinline__ float softplus(float x) {
+  return x > 20.0f ? x : log1pf(ex2_approx(x * kLog2e));
+}
+
+// Pack / unpack helpers for 16-byte vector access.
+union Pack16 {
+  uint4 u;
+  float f[4];
+  bf16 h[8];
+  __nv_bfloat162 h2[4];
+};
+
+}  // namespace sambay

@@ -1,0 +1,593 @@
+// libsambay: C ABI of the SambaY scan + Gated Memory Unit hot path on B200.
+// Host side: argument validation, workspace carving, TMA descriptors and
+// kernel launches.  Every step of the computation runs in the kernels of
+// scan_kernels.cuh, tc_gemm.cuh and simt_gemm.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/sambay.h"
+#include "common.cuh"
+#include "scan_kernels.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.cuh"
+
+using sambay::bf16;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------ device facts
+
+struct DeviceInfo {
+  int checked = 0;
+  int ok = 0;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+sambay_status current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAMBAY_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SAMBAY_ERR_DEVICE;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+    d.ok = (major == 10);
+    d.sms = sms;
+    d.checked = 1;
+  }
+  if (!d.ok) return SAMBAY_ERR_DEVICE;
+  *dev_out = dev;
+  *sms_out = d.sms;
+  return SAMBAY_OK;
+}
+
+// ------------------------------------------------------------ validation
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t io_bytes(int io) { return io == SAMBAY_BF16 ? 2 : 4; }
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+sambay_status check_dims(const sambay_dims* d, bool need_model, bool need_scan) {
+  if (!d) return SAMBAY_ERR_INVALID_ARG;
+  if (d->io != SAMBAY_F32 && d->io != SAMBAY_BF16) return SAMBAY_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->d_inner < 1) return SAMBAY_ERR_INVALID_ARG;
+  if (need_scan) {
+    if (d->seqlen < 1 || d->d_state < 1 || d->d_conv < 1 || d->dt_rank < 1)
+      return SAMBAY_ERR_INVALID_ARG;
+    if (d->d_state != 16 || d->d_conv != 4) return SAMBAY_ERR_UNSUPPORTED;
+    if (d->dt_rank % 4 != 0) return SAMBAY_ERR_UNSUPPORTED;
+    if (d->dt_rank + 2 * d->d_state > 256) return SAMBAY_ERR_UNSUPPORTED;
+    if (d->d_inner % 32 != 0) return SAMBAY_ERR_UNSUPPORTED;
+    if (d->io == SAMBAY_BF16 && (d->d_inner % 64 != 0 || d->dt_rank % 8 != 0))
+      return SAMBAY_ERR_UNSUPPORTED;
+  }
+  if (need_model) {
+    if (d->d_model < 1) return SAMBAY_ERR_INVALID_ARG;
+    if (d->io == SAMBAY_BF16 && (d->d_model % 64 != 0 || d->d_inner % 64 != 0))
+      return SAMBAY_ERR_UNSUPPORTED;
+    if (d->io == SAMBAY_F32 && (d->d_model % 4 != 0 || d->d_inner % 4 != 0))
+      return SAMBAY_ERR_UNSUPPORTED;
+  }
+  return SAMBAY_OK;
+}
+
+sambay_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return SAMBAY_ERR_INVALID_ARG;
+    if (!aligned16(p)) return SAMBAY_ERR_UNSUPPORTED;
+  }
+  return SAMBAY_OK;
+}
+
+sambay_status check_weights(const sambay_scan_weights* w) {
+  if (!w) return SAMBAY_ERR_INVALID_ARG;
+  return check_ptrs({w->conv_w, w->conv_b, w->x_proj_w, w->dt_proj_w, w->dt_bias, w->A, w->D});
+}
+
+sambay_status check_ws(const void* ws, size_t have, size_t need) {
+  if (need == 0) return SAMBAY_OK;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || have < need) return SAMBAY_ERR_WORKSPACE;
+  return SAMBAY_OK;
+}
+
+// ------------------------------------------------------------ workspace
+
+// Split-K factor of the tensor-core GEMMs that reduce over a long K with few
+// output tiles (x_proj, GMU decode).  A function of the sizes only, sized for
+// B200's 148 SMs, so the workspace and the summation order do not depend on
+// the device.
+constexpr int kSplitTarget = 148;
+
+int split_count(long long out_tiles, long long k, int max_splits) {
+  const long long k_blocks = (k + sambay::tc::BK - 1) / sambay::tc::BK;
+  long long s = std::max(1LL, kSplitTarget / std::max(1LL, out_tiles));
+  s = std::min<long long>(s, max_splits);
+  s = std::min(s, k_blocks);
+  const long long per = (k_blocks + s - 1) / s;  // k-blocks per split
+  return static_cast<int>((k_blocks + per - 1) / per);
+}
+
+constexpr int kXprojMaxSplits = 16;
+
+// bf16 mode: x_proj reduces over K = 2*Di (the split uc pair)
+int xproj_splits(long long rows, int d_inner) {
+  return split_count((rows + sambay::tc::BM - 1) / sambay::tc::BM, 2LL * d_inner, kXprojMaxSplits);
+}
+
+// dt_rank rounded up to whole 64-wide K blocks (each half of the split delta)
+int rank_pad(int R) { return (R + 63) / 64 * 64; }
+
+struct ScanWs {
+  size_t uc, part, xdbl, delta, dt, total;
+  int splits;
+};
+
+ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
+  ScanWs w{};
+  const long long Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
+  const bool tc = d->io == SAMBAY_BF16;
+  w.splits = tc ? xproj_splits(T, d->d_inner) : 1;
+  size_t off = 0;
+  // uc: f32, or the bf16 split pair (hi | lo): 4 bytes per element either way
+  w.uc = off;    off += round256(static_cast<size_t>(T * Di) * 4);
+  w.part = off;  off += tc ? round256(static_cast<size_t>(w.splits) * T * ldx * 4) : 0;
+  w.xdbl = off;  off += round256(static_cast<size_t>(T * ldx) * 4);
+  w.delta = off; off += tc ? round256(static_cast<size_t>(T) * 2 * rank_pad(static_cast<int>(R)) * 2) : 0;
+  w.dt = off;    off += round256(static_cast<size_t>(T * Di) * 4);
+  w.total = off;
+  return w;
+}
+
+struct GmuWs {
+  size_t h, part, counters, total;
+  int splits1, splits2;
+};
+
+constexpr int kStepMaxRows = 256;
+constexpr int kStepMaxSplits = 8;
+
+GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
+  GmuWs w{};
+  size_t off = 0;
+  w.h = off;
+  off += round256(static_cast<size_t>(rows) * d->d_inner * io_bytes(d->io));
+  if (step && d->io == SAMBAY_BF16) {
+    // swap-AB: output tiles run over d_inner (GEMM1) and d_model (GEMM2)
+    w.splits1 = split_count((d->d_inner + 127) / 128, d->d_model, kStepMaxSplits);
+    w.splits2 = split_count((d->d_model + 127) / 128, d->d_inner, kStepMaxSplits);
+    w.part = off;
+    off += round256(static_cast<size_t>(rows) *
+                    std::max(static_cast<long long>(w.splits1) * d->d_inner,
+                             static_cast<long long>(w.splits2) * d->d_model) * 4);
+    w.counters = off;
+    off += round256(static_cast<size_t>((d->d_inner + 127) / 128 + (d->d_model + 127) / 128) * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch row_bytes),
+// box {64 inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ tensor-core GEMM launch
+
+// An operand in memory: `rows` x `cols` bf16, cols contiguous.
+struct Operand {
+  const void* ptr;
+  long long rows, cols;
+};
+
+// `splits` > 1 splits K into that many contiguous ranges (as computed by
+// split_count for the same sizes).
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
+sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArgs g, int splits,
+                     cudaStream_t st) {
+  using namespace sambay::tc;
+  using C = Cfg<BN, A_MN, B_MN>;
+  static bool attr_set[kMaxDevices] = {};
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmem)) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  CUtensorMap ta, tb;
+  // A K-major: [M, K] -> box {64 k, 128 m};  MN-major: [K, M] -> box {64 m, 64 k}
+  if (!make_map(&ta, a.ptr, a.cols, a.rows, a.cols * 2, A_MN ? 64 : BM)) return SAMBAY_ERR_CUDA;
+  if (!make_map(&tb, b.ptr, b.cols, b.rows, b.cols * 2, B_MN ? 64 : BN)) return SAMBAY_ERR_CUDA;
+  g.m_tiles = (g.M + BM - 1) / BM;
+  g.n_tiles = (g.N + BN - 1) / BN;
+  g.k_blocks = (g.K + BK - 1) / BK;
+  splits = std::max(1, std::min(splits, g.k_blocks));
+  g.kb_per_split = (g.k_blocks + splits - 1) / splits;
+  g.splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
+  g.tiles = g.m_tiles * g.n_tiles * g.splits;
+  const int grid = std::min(g.tiles, sms);
+  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, g);
+  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+}
+
+sambay::tc::GemmArgs tc_args(int M, int N, int K, void* out, long long ldo, const void* aux = nullptr,
+                             const float* vec = nullptr, float* partials = nullptr,
+                             long long split_stride = 0, int* counters = nullptr) {
+  sambay::tc::GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.out = out;
+  g.aux = aux;
+  g.vec = vec;
+  g.ldo = ldo;
+  g.partials = partials;
+  g.split_stride = split_stride;
+  g.counters = counters;
+  return g;
+}
+
+// ------------------------------------------------------------ fp32 GEMM launch
+
+template <int KIND>
+sambay_status run_simt(const sambay::simt::Args& g, cudaStream_t st) {
+  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
+  sambay::simt::simt_gemm_kernel<KIND><<<grid, 256, 0, st>>>(g);
+  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+}
+
+sambay::simt::Args simt_args(const float* A, long long sam, long long sak, const float* B,
+                             long long sbk, long long sbn, int M, int N, int K, float* out,
+                             long long ldo, const float* aux = nullptr, const float* vec = nullptr) {
+  sambay::simt::Args g{};
+  g.A = A; g.sam = sam; g.sak = sak;
+  g.B = B; g.sbk = sbk; g.sbn = sbn;
+  g.M = M; g.N = N; g.K = K;
+  g.out = out; g.ldo = ldo; g.aux = aux; g.vec = vec; g.trans = 0;
+  return g;
+}
+
+#define SAMBAY_TRY(expr)                 \
+  do {                                   \
+    const sambay_status _s = (expr);     \
+    if (_s != SAMBAY_OK) return _s;      \
+  } while (0)
+
+int grid_for(long long threads, int block, int sms) {
+  const long long g = (threads + block - 1) / block;
+  return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(sms) * 16)));
+}
+
+// ------------------------------------------------------------ shared scan pieces
+
+// x_proj + dt_proj for `rows` tokens whose conv output is ws.uc:
+//   xdbl = uc W_x^T,  dt = softplus(delta W_dt^T + b_dt)
+sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
+                          long long rows, uint8_t* ws, const ScanWs& L, cudaStream_t st) {
+  const int Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
+  float* xdbl = reinterpret_cast<float*>(ws + L.xdbl);
+  float* dt = reinterpret_cast<float*>(ws + L.dt);
+  if (d->io == SAMBAY_BF16) {
+    const bf16* uc = reinterpret_cast<const bf16*>(ws + L.uc);
+    bf16* delta = reinterpret_cast<bf16*>(ws + L.delta);
+    float* part = reinterpret_cast<float*>(ws + L.part);
+    const long long stride = rows * ldx;
+    const int Rp = rank_pad(R);
+    // x_proj = [uc_hi | uc_lo] [W_x | W_x]^T, split over K: each split writes
+    // its partial [rows, ldx] tile set
+    auto gx = tc_args(static_cast<int>(rows), ldx, 2 * Di, part, ldx, nullptr, nullptr, nullptr, stride);
+    gx.b_k_wrap = Di;
+    const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
+    constexpr int P = sambay::tc::EPI_F32_PARTIAL;
+    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else SAMBAY_TRY((run_tc<256, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    sambay::scan::xdbl_reduce_kernel<<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
+        part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+    // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
+    // the A operand is padded with zeros to Rp, W_dt reads zeros past R
+    auto gd = tc_args(static_cast<int>(rows), Di, 2 * Rp, dt, Di, nullptr, w->dt_bias);
+    gd.b_k_wrap = Rp;
+    const Operand a_d{delta, rows, 2LL * Rp}, b_wdt{w->dt_proj_w, Di, R};
+    SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
+  } else {
+    const float* uc = reinterpret_cast<const float*>(ws + L.uc);
+    SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>(
+        simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
+                  ldx, Di, xdbl, ldx),
+        st));
+    SAMBAY_TRY(run_simt<sambay::simt::SOFTPLUS>(
+        simt_args(xdbl, ldx, 1, static_cast<const float*>(w->dt_proj_w), 1, R,
+                  static_cast<int>(rows), Di, R, dt, Di, nullptr, w->dt_bias),
+        st));
+  }
+  return SAMBAY_OK;
+}
+
+template <typename T>
+sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
+                                const sambay_dims* d, const void* u, void* M, float* ssm_state,
+                                void* conv_state, int zero_init, uint8_t* ws, cudaStream_t st) {
+  const long long T_ = static_cast<long long>(d->batch) * d->seqlen;
+  const ScanWs L = scan_ws_layout(d, T_);
+  T* uc = reinterpret_cast<T*>(ws + L.uc);
+  {
+    sambay::scan::ConvParams<T> p{static_cast<const T*>(u), static_cast<const T*>(conv_state),
+                                  static_cast<const T*>(w->conv_w),
+                                  static_cast<const T*>(w->conv_b), uc, d->batch, d->seqlen,
+                                  d->d_inner, zero_init};
+    constexpr int VEC = 16 / sizeof(T);
+    const long long threads =
+        static_cast<long long>(d->batch) * ((d->seqlen + 15) / 16) * (d->d_inner / VEC);
+    sambay::scan::conv_silu_kernel<T, 16><<<grid_for(threads, 256, sms), 256, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+  }
+  SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st));
+  {
+    sambay::scan::ScanParams<T> p{};
+    p.uc = uc;
+    p.dt = reinterpret_cast<const float*>(ws + L.dt);
+    p.xdbl = reinterpret_cast<const float*>(ws + L.xdbl);
+    p.A = w->A;
+    p.D = w->D;
+    p.u = static_cast<const T*>(u);
+    p.h = ssm_state;
+    p.conv_state = static_cast<T*>(conv_state);
+    p.M = static_cast<T*>(M);
+    p.B = d->batch;
+    p.L = d->seqlen;
+    p.Di = d->d_inner;
+    p.R = d->dt_rank;
+    p.ldx = d->dt_rank + 2 * d->d_state;
+    p.zero_init = zero_init;
+    dim3 grid(d->d_inner / sambay::scan::kScanCh, d->batch);
+    sambay::scan::selective_scan_kernel<T><<<grid, 128, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+  }
+  return SAMBAY_OK;
+}
+
+template <typename T>
+sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
+                             const void* u_t, void* m_t, float* ssm_state, void* conv_state,
+                             uint8_t* ws, cudaStream_t st) {
+  const long long B = d->batch;
+  const ScanWs L = scan_ws_layout(d, B);
+  T* uc = reinterpret_cast<T*>(ws + L.uc);
+  constexpr int VEC = 16 / sizeof(T);
+  sambay::scan::step_conv_kernel<T><<<grid_for(B * (d->d_inner / VEC), 256, 1 << 20), 256, 0, st>>>(
+      static_cast<const T*>(u_t), static_cast<T*>(conv_state), static_cast<const T*>(w->conv_w),
+      static_cast<const T*>(w->conv_b), uc, d->batch, d->d_inner);
+  if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+  SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st));
+  sambay::scan::step_scan_kernel<T><<<grid_for(B * d->d_inner * 4, 256, 1 << 20), 256, 0, st>>>(
+      uc, reinterpret_cast<const float*>(ws + L.dt), reinterpret_cast<const float*>(ws + L.xdbl),
+      w->A, w->D, ssm_state, static_cast<T*>(m_t), d->batch, d->d_inner, d->dt_rank,
+      d->dt_rank + 2 * d->d_state);
+  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ GMU
+
+sambay_status gmu_f32(const sambay_dims* d, long long rows, const void* X, const void* M,
+                      const void* W1, const void* W2, const void* residual, void* Y, uint8_t* ws,
+                      const GmuWs& L, cudaStream_t st) {
+  const int Dm = d->d_model, Di = d->d_inner;
+  float* H = reinterpret_cast<float*>(ws + L.h);
+  SAMBAY_TRY(run_simt<sambay::simt::GATE>(
+      simt_args(static_cast<const float*>(X), Dm, 1, static_cast<const float*>(W1), 1, Dm,
+                static_cast<int>(rows), Di, Dm, H, Di, static_cast<const float*>(M)),
+      st));
+  SAMBAY_TRY(run_simt<sambay::simt::RESID>(
+      simt_args(H, Di, 1, static_cast<const float*>(W2), Dm, 1, static_cast<int>(rows), Dm, Di,
+                static_cast<float*>(Y), Dm, static_cast<const float*>(residual)),
+      st));
+  return SAMBAY_OK;
+}
+
+sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                                const void* W1, const void* W2, const void* residual, void* Y) {
+  SAMBAY_TRY(check_dims(d, true, false));
+  if (rows < 1 || rows > (1LL << 30)) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({X, M, W1, W2, Y}));
+  if (residual && !aligned16(residual)) return SAMBAY_ERR_UNSUPPORTED;
+  if (Y == M || (Y == X && X != residual)) return SAMBAY_ERR_INVALID_ARG;
+  return SAMBAY_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* sambay_status_string(sambay_status s) {
+  switch (s) {
+    case SAMBAY_OK: return "ok";
+    case SAMBAY_ERR_INVALID_ARG: return "invalid argument";
+    case SAMBAY_ERR_UNSUPPORTED: return "unsupported size or alignment";
+    case SAMBAY_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SAMBAY_ERR_CUDA: return "CUDA call failed";
+    case SAMBAY_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case SAMBAY_ERR_DEVICE: return "no sm_100 device current";
+  }
+  return "unknown status";
+}
+
+const char* sambay_version(void) { return "0.1.0"; }
+
+size_t sambay_scan_prefill_workspace(const sambay_dims* d) {
+  if (check_dims(d, false, true) != SAMBAY_OK) return 0;
+  return scan_ws_layout(d, static_cast<long long>(d->batch) * d->seqlen).total;
+}
+
+size_t sambay_scan_step_workspace(const sambay_dims* d) {
+  if (!d) return 0;
+  sambay_dims e = *d;
+  e.seqlen = 1;
+  if (check_dims(&e, false, true) != SAMBAY_OK) return 0;
+  return scan_ws_layout(&e, e.batch).total;
+}
+
+size_t gmu_forward_workspace(const sambay_dims* d, int64_t rows) {
+  if (check_dims(d, true, false) != SAMBAY_OK || rows < 1) return 0;
+  return gmu_ws_layout(d, rows, false).total;
+}
+
+size_t gmu_step_workspace(const sambay_dims* d, int64_t rows) {
+  if (check_dims(d, true, false) != SAMBAY_OK || rows < 1 || rows > kStepMaxRows) return 0;
+  return gmu_ws_layout(d, rows, true).total;
+}
+
+sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const sambay_dims* d, const void* u,
+                                  void* M, float* ssm_state, void* conv_state, int zero_init_state,
+                                  void* ws, size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, false, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u, M, ssm_state, conv_state}));
+  if (M == u) return SAMBAY_ERR_INVALID_ARG;
+  const size_t need = sambay_scan_prefill_workspace(d);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, need));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int zi = zero_init_state ? 1 : 0;
+  if (d->io == SAMBAY_BF16)
+    return scan_prefill_impl<bf16>(dev, sms, w, d, u, M, ssm_state, conv_state, zi, w8, st);
+  return scan_prefill_impl<float>(dev, sms, w, d, u, M, ssm_state, conv_state, zi, w8, st);
+}
+
+sambay_status sambay_scan_step(const sambay_scan_weights* w, const sambay_dims* d, const void* u_t,
+                               void* m_t, float* ssm_state, void* conv_state, void* ws,
+                               size_t ws_bytes, sambay_stream_t stream) {
+  if (!d) return SAMBAY_ERR_INVALID_ARG;
+  sambay_dims e = *d;
+  e.seqlen = 1;
+  SAMBAY_TRY(check_dims(&e, false, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u_t, m_t, ssm_state, conv_state}));
+  if (m_t == u_t) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_scan_step_workspace(&e)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (e.io == SAMBAY_BF16)
+    return scan_step_impl<bf16>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
+  return scan_step_impl<float>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
+}
+
+sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                          const void* W1, const void* W2, const void* residual, void* Y, void* ws,
+                          size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(gmu_common_checks(d, rows, X, M, W1, W2, residual, Y));
+  const GmuWs L = gmu_ws_layout(d, rows, false);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, residual, Y, w8, L, st);
+  const int Dm = d->d_model, Di = d->d_inner, T = static_cast<int>(rows);
+  bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
+  // G = X W1^T, epilogue H = M ⊙ SiLU(G)
+  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false>(
+      dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st)));
+  // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
+  SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false>(
+      dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
+      st)));
+  return SAMBAY_OK;
+}
+
+sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                       const void* W1, const void* W2, const void* residual, void* Y, void* ws,
+                       size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(gmu_common_checks(d, rows, X, M, W1, W2, residual, Y));
+  if (rows > kStepMaxRows) return SAMBAY_ERR_UNSUPPORTED;
+  const GmuWs L = gmu_ws_layout(d, rows, true);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, residual, Y, w8, L, st);
+  const int Dm = d->d_model, Di = d->d_inner, Bn = static_cast<int>(rows);
+  bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
+  float* part = reinterpret_cast<float*>(w8 + L.part);
+  int* counters = reinterpret_cast<int*>(w8 + L.counters);
+  // split-K arrival counters start at zero; the last CTA of each tile resets
+  // its counter, so the second GEMM finds them zero again
+  if (cudaMemsetAsync(counters, 0, L.total - L.counters, st) != cudaSuccess) return SAMBAY_ERR_CUDA;
+  // swap-AB: H^T = SiLU(W1 X^T) ⊙ M^T; W1 rows stream once through the tensor cores
+  const auto g1 = tc_args(Di, Bn, Dm, H, Di, M, nullptr, part, rows * static_cast<long long>(Di), counters);
+  const auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual, nullptr, part, rows * static_cast<long long>(Dm), counters);
+  const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
+#define SAMBAY_STEP_GEMMS(BNV)                                                                   \
+  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>(dev, sms, w1, xr, g1, L.splits1, st))); \
+  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>(dev, sms, w2, hr, g2, L.splits2, st)));
+  if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
+  else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
+  else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }
+  else { SAMBAY_STEP_GEMMS(256) }
+#undef SAMBAY_STEP_GEMMS
+  return SAMBAY_OK;
+}
+
+sambay_status sambay_device_status(sambay_stream_t stream, int32_t* out_code) {
+  if (!out_code) return SAMBAY_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SAMBAY_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, sambay::g_status, sizeof(int)) != cudaSuccess) return SAMBAY_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(sambay::g_status, &zero, sizeof(int)) != cudaSuccess) return SAMBAY_ERR_CUDA;
+  *out_code = v;
+  return SAMBAY_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,552 @@
+// Persistent tcgen05 (5th-gen tensor core) GEMM for sm_100a, bf16 in, fp32
+// accumulate in TMEM, operands staged in shared memory by TMA, with fused
+// epilogues.  One CTA per SM; warp roles:
+//   warp 0        TMA producer (one lane): A and B tiles into a smem ring
+//   warp 1        MMA issuer (one lane) + TMEM owner (whole warp allocates)
+//   warps 2..5    epilogue: tcgen05.ld TMEM -> registers -> fused op -> HBM
+// The accumulator is double-buffered in TMEM so the epilogue of one tile
+// overlaps the main loop of the next.  No cluster multicast is used: every
+// CTA loads its own tiles.
+//
+// D[m, n] = sum_k A[m, k] * B[k, n]
+//   A: K-major ([M, K], k contiguous) or MN-major ([K, M], m contiguous)
+//   B: K-major ([N, K], k contiguous) or MN-major ([K, N], n contiguous)
+// Tile 128 x BN x 64, SWIZZLE_128B smem layout (what TMA writes with a 128-byte
+// inner box), UMMA smem descriptors per the sm_100 matrix-descriptor format.
+//
+// Every mbarrier wait is bounded (clock64); on expiry the kernel records
+// SAMBAY_ERR_TIMEOUT in the device status word, raises a CTA-wide abort flag,
+// drains its in-flight TMA loads and MMAs (again bounded), frees TMEM and
+// returns.
+#pragma once
+
+#include <cuda.h>
+#include "common.cuh"
+
+namespace sambay {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                       // one 128-byte swizzle atom of bf16
+constexpr int kThreads = 192;                // 6 warps
+constexpr unsigned long long kWaitCycles = 1ull << 34;  // ~8 s at 2 GHz
+constexpr unsigned long long kDrainCycles = 1ull << 28;
+
+// ------------------------------------------------------------------ PTX glue
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait.  Returns false if the CTA is aborting (flag already raised by
+// another role) or this wait ran out (then it raises the flag itself).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit = kWaitCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (static_cast<unsigned long long>(clock64() - t0) > limit) {
+      *abort_flag = 1;
+      record_status(kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp receives row
+// (lane base + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// AND of a predicate over the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ bool epi_agree(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
+// Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 format (version 1).
+//   K-major : 8-row x 128-byte atoms; SBO = 1024 B between 8-row groups.
+//   MN-major: 64-element x 8-row atoms; LBO = stride between 64-element MN
+//             groups, SBO = 1024 B between 8-row K groups.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= 1ull << 46;  // descriptor version (sm_100)
+  d |= 2ull << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                       // D format: f32
+         | (1u << 7)                     // A format: bf16
+         | (1u << 10)                    // B format: bf16
+         | ((a_mn ? 1u : 0u) << 15)      // A major
+         | ((b_mn ? 1u : 0u) << 16)      // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- epilogues
+
+enum EpiKind : int {
+  EPI_F32_PARTIAL = 0,  // out(f32)[split][...] = acc     (split-K partials, summed by the caller)
+  EPI_GATE = 1,      // out(bf16) = SiLU(acc) * aux      (GMU gate: H = M ⊙ SiLU(X W1^T))
+  EPI_RESID = 2,     // out(bf16) = acc (+ aux if given)  (GMU output + residual)
+  EPI_SOFTPLUS = 3,  // out(f32) = softplus(acc + vec[n]) (dt_proj)
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int m_tiles, n_tiles, splits, kb_per_split, k_blocks, tiles;
+  void* out;          // output base
+  const void* aux;    // EPI_GATE: memory readout M; EPI_RESID: residual or NULL
+  const float* vec;   // EPI_SOFTPLUS: per-column bias
+  long long ldo;      // leading dimension (elements) of out and aux
+  long long split_stride;  // elements between consecutive splits' partials
+  float* partials;    // split-K partial tiles [splits][split_stride] (f32)
+  int* counters;      // split-K arrival counters per (m, n) tile, zero on entry
+  int b_k_wrap;       // > 0: B's k coordinate wraps at this multiple of 64, so an A
+                      // of [hi | lo] halves meets the same B twice (split-bf16 operand)
+};
+
+// The final op on one element.  `o` is the output's linear index.
+template <int KIND>
+__device__ __forceinline__ void epi_store_one(const GemmArgs& g, long long o, int n, float v) {
+  if (KIND == EPI_F32_PARTIAL) {
+    reinterpret_cast<float*>(g.out)[o] = v;
+  } else if (KIND == EPI_GATE) {
+    const float m = to_f32(reinterpret_cast<const bf16*>(g.aux)[o]);
+    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(silu(v) * m);
+  } else if (KIND == EPI_RESID) {
+    const float r = g.aux ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o]) : 0.0f;
+    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(v + r);
+  } else {
+    reinterpret_cast<float*>(g.out)[o] = softplus(v + g.vec[n]);
+  }
+}
+
+// One thread's 32 accumulator values of row `m`, columns [n0, n0 + 32).
+// TRANS: the output is stored transposed, out[n * ldo + m] (swap-AB GEMV).
+template <int KIND, bool TRANS>
+__device__ __forceinline__ void epi_chunk(const GemmArgs& g, int m, int n0, const float (&v)[32]) {
+  if (m >= g.M) return;
+  if (!TRANS && n0 + 32 <= g.N && (g.ldo % 8) == 0) {
+    // vectorised row segment: 32 contiguous outputs
+    const long long base = static_cast<long long>(m) * g.ldo + n0;
+    if (KIND == EPI_F32_PARTIAL) {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + base);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else if (KIND == EPI_SOFTPLUS) {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + base);
+      const float4* bias = reinterpret_cast<const float4*>(g.vec + n0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 b = bias[j];
+        float4 r;
+        r.x = softplus(v[4 * j + 0] + b.x);
+        r.y = softplus(v[4 * j + 1] + b.y);
+        r.z = softplus(v[4 * j + 2] + b.z);
+        r.w = softplus(v[4 * j + 3] + b.w);
+        dst[j] = r;
+      }
+    } else {
+      const uint4* auxv = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(g.aux) + base);
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        Pack16 a, r;
+        if (KIND == EPI_GATE || g.aux) a.u = auxv[j];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = v[8 * j + 2 * e], x1 = v[8 * j + 2 * e + 1];
+          float y0, y1;
+          if (KIND == EPI_GATE) {
+            const float2 mm = __bfloat1622float2(a.h2[e]);
+            y0 = silu(x0) * mm.x;
+            y1 = silu(x1) * mm.y;
+          } else if (g.aux) {
+            const float2 rr = __bfloat1622float2(a.h2[e]);
+            y0 = x0 + rr.x;
+            y1 = x1 + rr.y;
+          } else {
+            y0 = x0;
+            y1 = x1;
+          }
+          r.h2[e] = __floats2bfloat162_rn(y0, y1);
+        }
+        dst[j] = r.u;
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int n = n0 + j;
+    if (n < g.N) {
+      const long long o = TRANS ? static_cast<long long>(n) * g.ldo + m
+                                : static_cast<long long>(m) * g.ldo + n;
+      epi_store_one<KIND>(g, o, n, v[j]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int BN, bool A_MN, bool B_MN>
+struct Cfg {
+  static constexpr int kABytes = BM * BK * 2;   // 16 KB
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+  static constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
+  static constexpr size_t kSmem = 1024 /*align slack*/ + static_cast<size_t>(kStages) * kStageBytes + 256;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element atoms");
+};
+
+struct TileCoord {
+  int m, n, split, kb0, kb1;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
+  TileCoord c;
+  c.m = t % g.m_tiles;
+  const int r = t / g.m_tiles;
+  c.n = r % g.n_tiles;
+  c.split = r / g.n_tiles;
+  c.kb0 = c.split * g.kb_per_split;
+  c.kb1 = min(g.k_blocks, c.kb0 + g.kb_per_split);
+  return c;
+}
+
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs g) {
+  using C = Cfg<BN, A_MN, B_MN>;
+  constexpr int S = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;      // [2]
+  uint64_t* tempty = tfull + 2;     // [2]
+  uint64_t* drain = tempty + 2;     // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;  // per stage: outstanding load, its parity
+      bool ok = true;
+      for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
+        const TileCoord c = tile_coord(g, t);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          uint8_t* a_dst = sA + stage * C::kABytes;
+          uint8_t* b_dst = sB + stage * C::kBBytes;
+          if (A_MN) {  // [K, M] in memory: boxes of 64 m x 64 k
+            tma_load_2d(a_dst, &tmA, &full[stage], c.m * BM, kb * BK);
+            tma_load_2d(a_dst + 8192, &tmA, &full[stage], c.m * BM + 64, kb * BK);
+          } else {     // [M, K]: one box of 64 k x 128 m
+            tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, c.m * BM);
+          }
+          const int kb_b = g.b_k_wrap > 0 ? (kb * BK) % g.b_k_wrap : kb * BK;
+          if (B_MN) {  // [K, N]: BN/64 boxes of 64 n x 64 k
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(b_dst + j * 8192, &tmB, &full[stage], c.n * BN + 64 * j, kb_b);
+          } else {     // [N, K]: one box of 64 k x BN n
+            tma_load_2d(b_dst, &tmB, &full[stage], kb_b, c.n * BN);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // drain: every issued load must land before the CTA's smem goes away
+        for (int s = 0; s < S; ++s)
+          if (issued_mask & (1u << s)) {
+            volatile int dummy = 0;
+            mbar_wait(&full[s], (issued_parity >> s) & 1u, &dummy, kDrainCycles);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
+        const TileCoord c = tile_coord(g, t);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                     : sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                     : sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, C::kIdesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all MMAs issued by this thread complete before TMEM is released
+      tc_commit(drain);
+      volatile int dummy = 0;
+      mbar_wait(drain, 0, &dummy, kDrainCycles);
+    }
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int quarter = warp & 3;            // TMEM lanes [32*quarter, +32)
+    const int ep_tid = threadIdx.x - 64;     // 0..127
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < g.tiles; t += gridDim.x) {
+      const TileCoord c = tile_coord(g, t);
+      const bool split = g.splits > 1 && KIND != EPI_F32_PARTIAL;
+      bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      // the split-K path synchronises the 4 epilogue warps, so they must agree
+      // on leaving the loop together
+      if (split) ok = epi_agree(ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = c.m * BM + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + ch * 32, r);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        const int n0 = c.n * BN + ch * 32;
+        if (split) {
+          // this split's partial tile, summed in split order by the last CTA
+          float* part = g.partials + static_cast<long long>(c.split) * g.split_stride;
+          if (row < g.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int n = n0 + j;
+              if (n < g.N) {
+                const long long o = TRANS ? static_cast<long long>(n) * g.ldo + row
+                                          : static_cast<long long>(row) * g.ldo + n;
+                __stcg(part + o, v[j]);
+              }
+            }
+          }
+        } else if (KIND == EPI_F32_PARTIAL) {
+          GemmArgs gs = g;
+          gs.out = reinterpret_cast<float*>(g.out) + static_cast<long long>(c.split) * g.split_stride;
+          epi_chunk<KIND, TRANS>(gs, row, n0, v);
+        } else {
+          epi_chunk<KIND, TRANS>(g, row, n0, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+
+      if (split) {
+        // The last CTA to finish a split-K tile sums the partials in split
+        // order (deterministic), applies the final op and resets the counter.
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ep_tid == 0) {
+          const int tile_mn = c.m + g.m_tiles * c.n;
+          const int prev = atomicAdd(g.counters + tile_mn, 1);
+          const int last = (prev == g.splits - 1);
+          if (last) g.counters[tile_mn] = 0;
+          *last_flag = last;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (*last_flag) {
+          __threadfence();
+          if (row < g.M) {
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+              const int n0 = c.n * BN + ch * 32;
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int n = n0 + j;
+                v[j] = 0.0f;
+                if (n < g.N) {
+                  const long long o = TRANS ? static_cast<long long>(n) * g.ldo + row
+                                            : static_cast<long long>(row) * g.ldo + n;
+                  float acc = 0.0f;
+                  for (int sp = 0; sp < g.splits; ++sp)
+                    acc += __ldcg(g.partials + static_cast<long long>(sp) * g.split_stride + o);
+                  v[j] = acc;
+                }
+              }
+              epi_chunk<KIND, TRANS>(g, row, n0, v);
+            }
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace tc
+}  // namespace sambay

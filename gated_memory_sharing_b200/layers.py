@@ -1,0 +1,135 @@
+"""Device-resident layers over the C ABI: a Mamba scan layer that produces the
+memory readout M, and Gated Memory Units that reuse it.
+
+These hold the weights and workspaces in torch-allocated device memory and
+call the ABI entry points; they do no arithmetic of their own.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import abi
+
+
+def io_dtype(io: int) -> torch.dtype:
+    return torch.bfloat16 if io == abi.BF16 else torch.float32
+
+
+def to_device(a, io: int, device="cuda") -> torch.Tensor:
+    """float32 numpy array (already rounded to the I/O type) -> device tensor."""
+    return torch.from_numpy(a).to(device=device).to(io_dtype(io)).contiguous()
+
+
+def to_device_f32(a, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(a).to(device=device, dtype=torch.float32).contiguous()
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+class ScanLayer:
+    """The Mamba layer whose readout is the shared memory M."""
+
+    def __init__(self, w: dict, d_model: int, io: int, device="cuda"):
+        self.io = io
+        self.dtype = io_dtype(io)
+        self.d_inner, self.d_state = w["A"].shape
+        self.d_conv = w["conv_w"].shape[1]
+        self.dt_rank = w["dt_rank"]
+        self.d_model = d_model
+        self.conv_w = to_device(w["conv_w"], io, device)
+        self.conv_b = to_device(w["conv_b"], io, device)
+        self.x_proj_w = to_device(w["x_proj_w"], io, device)
+        self.dt_proj_w = to_device(w["dt_proj_w"], io, device)
+        self.dt_bias = to_device_f32(w["dt_bias"], device)
+        self.A = to_device_f32(w["A"], device)
+        self.D = to_device_f32(w["D"], device)
+        self.abi_w = abi.make_weights(self.conv_w, self.conv_b, self.x_proj_w, self.dt_proj_w,
+                                      self.dt_bias, self.A, self.D)
+        self.device = device
+        self._ws = {}
+
+    def dims(self, batch: int, seqlen: int) -> abi.Dims:
+        return abi.make_dims(batch, seqlen, self.d_model, self.d_inner, self.d_state, self.d_conv,
+                             self.dt_rank, self.io)
+
+    def _workspace(self, key, nbytes):
+        ws = self._ws.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = workspace(nbytes, self.device)
+            self._ws[key] = ws
+        return ws
+
+    def new_state(self, batch: int):
+        h = torch.zeros(batch, self.d_inner, self.d_state, dtype=torch.float32, device=self.device)
+        cs = torch.zeros(batch, self.d_inner, self.d_conv, dtype=self.dtype, device=self.device)
+        return h, cs
+
+    def prefill(self, u, ssm_state=None, conv_state=None, M=None, fresh=None, stream=None):
+        """u [B, L, Di] -> M [B, L, Di].  Without states (or with fresh=True)
+        the prompt starts from zero state; otherwise it continues the given
+        states.  States are returned and updated in place."""
+        B, L, _ = u.shape
+        if fresh is None:
+            fresh = ssm_state is None
+        if ssm_state is None:
+            ssm_state, conv_state = self.new_state(B)
+        if M is None:
+            M = torch.empty_like(u)
+        d = self.dims(B, L)
+        ws = self._workspace(("prefill", B, L), abi.sambay_scan_prefill_workspace(d))
+        abi.sambay_scan_prefill(self.abi_w, d, u, M, ssm_state, conv_state, fresh, ws, stream)
+        return M, ssm_state, conv_state
+
+    def step(self, u_t, ssm_state, conv_state, m_t=None, stream=None):
+        """u_t [B, Di] -> m_t [B, Di]; states updated in place."""
+        B = u_t.shape[0]
+        if m_t is None:
+            m_t = torch.empty_like(u_t)
+        d = self.dims(B, 1)
+        ws = self._workspace(("step", B), abi.sambay_scan_step_workspace(d))
+        abi.sambay_scan_step(self.abi_w, d, u_t, m_t, ssm_state, conv_state, ws, stream)
+        return m_t
+
+
+class GMULayer:
+    """Y = (M ⊙ SiLU(X W1^T)) W2 (+ X)."""
+
+    def __init__(self, W1, W2, io: int, device="cuda"):
+        self.io = io
+        self.W1 = to_device(W1, io, device)
+        self.W2 = to_device(W2, io, device)
+        self.d_inner, self.d_model = W1.shape
+        self.device = device
+        self._ws = {}
+
+    def dims(self, rows: int) -> abi.Dims:
+        return abi.make_dims(rows, 1, self.d_model, self.d_inner, 16, 4, 4, self.io)
+
+    def _workspace(self, key, nbytes):
+        ws = self._ws.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = workspace(nbytes, self.device)
+            self._ws[key] = ws
+        return ws
+
+    def forward(self, X, M, residual=False, Y=None, stream=None):
+        rows = X.shape[0]
+        if Y is None:
+            Y = torch.empty_like(X)
+        d = self.dims(rows)
+        ws = self._workspace(("fwd", rows), abi.gmu_forward_workspace(d, rows))
+        abi.gmu_forward(d, rows, X, M, self.W1, self.W2, X if residual else None, Y, ws, stream)
+        return Y
+
+    def step(self, X, M, residual=False, Y=None, stream=None):
+        rows = X.shape[0]
+        if Y is None:
+            Y = torch.empty_like(X)
+        d = self.dims(rows)
+        ws = self._workspace(("step", rows), abi.gmu_step_workspace(d, rows))
+        abi.gmu_step(d, rows, X, M, self.W1, self.W2, X if residual else None, Y, ws, stream)
+        return Y

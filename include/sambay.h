@@ -1,0 +1,191 @@
+/*
+ * sambay.h - C ABI of the SambaY scan + Gated Memory Unit hot path on B200
+ * (sm_100a).  Exported by libsambay.so.
+ *
+ * The method (sources cited per entry point):
+ *   [GMU]   "Decoder-Hybrid-Decoder Architecture for Efficient Reasoning with
+ *           Long Generation", Paper-Notes page, 方法详解 > 关键设计 (Gated Memory
+ *           Unit): Y = (M ⊙ SiLU(X W1^T)) W2, where M is the token-mixing output
+ *           of the self-decoder's last SSM layer, and decoding keeps a
+ *           constant-size recurrent state.
+ *   [FRAME] same page, 方法详解 > 整体框架: prefill runs only the self-decoder
+ *           (linear in length); the cross-decoder's GMU layers reuse M; a GMU
+ *           layer moves O(d_h) memory per decoded token.
+ *   [ABS]   the paper's abstract (chatpaper.ai page, English abstract): GMUs
+ *           share the "memory readout states" of the Samba self-decoder.
+ *   [MAMBA] the selective SSM producing M (Gu & Dao 2023, "Mamba", section
+ *           3.2 and Algorithm 2; block of section 3.4): causal depthwise
+ *           conv + SiLU, x_proj -> (delta, B, C), dt = softplus(delta W_dt^T +
+ *           b_dt), h_t = exp(dt A) h_{t-1} + dt B_t u_t, y_t = C_t h_t + D u_t.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers, caller-owned, row-major and
+ *     densely packed in the stated shape; the library allocates no device
+ *     memory and keeps no state between calls.  Scratch memory is the
+ *     caller's `ws` buffer of at least the queried size (256-byte aligned).
+ *   - "io" is the I/O element type of the call (dims->io): SAMBAY_F32 (float)
+ *     or SAMBAY_BF16 (bfloat16).  State, dt, B, C and every accumulation are
+ *     float32 in both modes.  SAMBAY_F32 runs float32 CUDA-core kernels
+ *     (no TF32); SAMBAY_BF16 runs the tcgen05 tensor-core kernels.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise, except sambay_device_status.
+ *   - Argument errors (NULL pointers, bad or unsupported sizes, misaligned
+ *     pointers, short workspace) are detected on the host BEFORE any launch,
+ *     and return a status without touching the device.  Launch failures
+ *     return SAMBAY_ERR_CUDA.  Faults found by a kernel while running (a
+ *     bounded wait that ran out) are recorded in a per-device status word
+ *     that sambay_device_status reads and clears.
+ *   - Supported sizes: d_state == 16, d_conv == 4, dt_rank a multiple of 4
+ *     with dt_rank + 2*d_state <= 256, d_inner a multiple of 32 (scan) or 4
+ *     (GMU), d_model a multiple of 4; in SAMBAY_BF16 mode d_inner and d_model
+ *     are multiples of 64 and dt_rank a multiple of 8 (16-byte rows for TMA).
+ *     batch, seqlen, rows >= 1; gmu_step rows <= 256.  Device pointers must
+ *     be 16-byte aligned (ws: 256-byte).  Anything else returns
+ *     SAMBAY_ERR_UNSUPPORTED (SAMBAY_ERR_INVALID_ARG for values < 1).
+ */
+#ifndef SAMBAY_H_
+#define SAMBAY_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SAMBAY_API __attribute__((visibility("default")))
+#else
+#define SAMBAY_API
+#endif
+
+typedef struct CUstream_st* sambay_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  SAMBAY_OK = 0,
+  SAMBAY_ERR_INVALID_ARG = 1, /* NULL pointer, non-positive size, bad enum    */
+  SAMBAY_ERR_UNSUPPORTED = 2, /* valid but outside the supported sizes above  */
+  SAMBAY_ERR_WORKSPACE = 3,   /* ws NULL/misaligned or ws_bytes too small     */
+  SAMBAY_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed            */
+  SAMBAY_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (device word) */
+  SAMBAY_ERR_DEVICE = 6       /* no sm_100 device current                     */
+} sambay_status;
+
+typedef enum { SAMBAY_F32 = 0, SAMBAY_BF16 = 1 } sambay_dtype;
+
+/* Sizes.  B batch, L seqlen, Dm d_model, Di d_inner, N d_state, K d_conv,
+ * R dt_rank.  T = B*L tokens. */
+typedef struct {
+  int32_t batch;
+  int32_t seqlen;
+  int32_t d_model;
+  int32_t d_inner;
+  int32_t d_state;
+  int32_t d_conv;
+  int32_t dt_rank;
+  int32_t io; /* sambay_dtype */
+} sambay_dims;
+
+/* Weights of the Mamba layer whose readout is M [MAMBA].  Device pointers. */
+typedef struct {
+  const void* conv_w;    /* [Di, K] io   depthwise causal conv taps; tap K-1
+                            multiplies the current token (cross-correlation) */
+  const void* conv_b;    /* [Di]    io   conv bias                           */
+  const void* x_proj_w;  /* [R+2N, Di] io rows [0,R): delta, [R,R+N): B,
+                            [R+N,R+2N): C                                    */
+  const void* dt_proj_w; /* [Di, R] io                                       */
+  const float* dt_bias;  /* [Di]    f32                                      */
+  const float* A;        /* [Di, N] f32  (negative; the decay is exp(dt*A))  */
+  const float* D;        /* [Di]    f32  skip weight                         */
+} sambay_scan_weights;
+
+/* ---------------------------------------------------------------------- */
+/* Workspace queries: bytes of caller-provided scratch each call needs.    */
+/* 0 on invalid dims.  Sizes depend only on the arguments.                 */
+/* ---------------------------------------------------------------------- */
+SAMBAY_API size_t sambay_scan_prefill_workspace(const sambay_dims* dims);
+SAMBAY_API size_t sambay_scan_step_workspace(const sambay_dims* dims);
+SAMBAY_API size_t gmu_forward_workspace(const sambay_dims* dims, int64_t rows);
+SAMBAY_API size_t gmu_step_workspace(const sambay_dims* dims, int64_t rows);
+
+/*
+ * sambay_scan_prefill - one Mamba selective scan over a prompt, writing the
+ * memory readout M and leaving the constant-size decode state [MAMBA],
+ * [GMU] (M^(l') = the token-mixing output; decode state), [FRAME] (prefill
+ * = self-decoder only), [ABS] ("memory readout states").
+ *
+ *   u          [B, L, Di] io  in   scan input (the in_proj x branch)
+ *   M          [B, L, Di] io  out  y = C.h + D*uc, before any output gate,
+ *                                  norm or out_proj.  Must not alias u.
+ *   ssm_state  [B, Di, N] f32 in/out  h; read as h_0 unless zero_init_state,
+ *                                  overwritten with h_L.
+ *   conv_state [B, Di, K] io  in/out  the last K scan inputs, oldest first;
+ *                                  read as left context unless
+ *                                  zero_init_state (then zeros), overwritten
+ *                                  with the last K inputs seen.
+ *   zero_init_state  nonzero: fresh prompt (states treated as zero).
+ *   ws, ws_bytes     scratch, >= sambay_scan_prefill_workspace(dims).
+ * Steps: uc = SiLU(conv(u)); [delta|B|C] = uc W_x^T; dt = softplus(delta
+ * W_dt^T + b_dt); the exp(dt A) recurrence with float32 h; readout.
+ */
+SAMBAY_API sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const sambay_dims* dims,
+                                  const void* u, void* M, float* ssm_state, void* conv_state,
+                                  int zero_init_state, void* ws, size_t ws_bytes,
+                                  sambay_stream_t stream);
+
+/*
+ * sambay_scan_step - one decode token per sequence: the prefill with L = 1
+ * on the carried state, updating ssm_state and conv_state IN PLACE [GMU]
+ * (constant-size state), [MAMBA].  dims->seqlen is ignored.
+ *
+ *   u_t [B, Di] io in;  m_t [B, Di] io out (must not alias u_t);
+ *   ssm_state [B, Di, N] f32 in/out;  conv_state [B, Di, K] io in/out.
+ */
+SAMBAY_API sambay_status sambay_scan_step(const sambay_scan_weights* w, const sambay_dims* dims,
+                               const void* u_t, void* m_t, float* ssm_state, void* conv_state,
+                               void* ws, size_t ws_bytes, sambay_stream_t stream);
+
+/*
+ * gmu_forward - Gated Memory Unit over `rows` tokens [GMU]:
+ *     Y = (M ⊙ SiLU(X W1^T)) W2   (+ residual when residual != NULL)
+ *
+ *   X  [rows, Dm] io   W1 [Di, Dm] io (used as W1^T)   M [rows, Di] io
+ *   W2 [Di, Dm] io (multiplies on the right: Di -> Dm)
+ *   residual [rows, Dm] io or NULL;  Y [rows, Dm] io out (may alias
+ *   residual, must not alias X unless X == residual, nor M).
+ * Two tensor-core GEMMs: G = X W1^T with SiLU(G) ⊙ M fused into its
+ * epilogue (H, io, kept in ws), then H W2 with the residual fused.
+ */
+SAMBAY_API sambay_status gmu_forward(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
+                          const void* W1, const void* W2, const void* residual, void* Y,
+                          void* ws, size_t ws_bytes, sambay_stream_t stream);
+
+/*
+ * gmu_step - the GMU for one decode token of `rows` sequences (rows <= 256)
+ * [GMU], [FRAME] (O(d_h) memory per token: the weights are streamed once).
+ * Same arguments and semantics as gmu_forward; a weight-streaming kernel
+ * pair (swap-AB tensor-core GEMV with split-K) instead of the tiled GEMMs.
+ */
+SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
+                       const void* W1, const void* W2, const void* residual, void* Y,
+                       void* ws, size_t ws_bytes, sambay_stream_t stream);
+
+/*
+ * sambay_device_status - synchronise `stream`, then read and clear the
+ * current device's status word.  *out_code receives the sambay_status a
+ * kernel recorded (SAMBAY_OK if none).  Returns SAMBAY_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+SAMBAY_API sambay_status sambay_device_status(sambay_stream_t stream, int32_t* out_code);
+
+/* Static, human-readable name of a status code. */
+SAMBAY_API const char* sambay_status_string(sambay_status status);
+
+/* Library version, "major.minor.patch". */
+SAMBAY_API const char* sambay_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* SAMBAY_H_ */

@@ -1,0 +1,190 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every symbol include/sambay.h declares; the
+workspace queries and status strings are pure host functions; and every
+argument error is reported before the library touches a device.  The error
+cases below are all built so that validation fails, so no call here can reach
+a kernel launch even on a GPU machine.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_memory_sharing_b200 import abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load()
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names.update(re.findall(r"^SAMBAY_API\s+[^;(]*?\b(\w+)\s*\(", src, re.M))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_symbols()
+    assert declared == set(abi.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), f"libsambay does not export {name}"
+
+
+def test_status_strings_and_version(lib):
+    assert abi.sambay_version() == "0.1.0"
+    assert abi.sambay_status_string(0) == "ok"
+    for code in range(1, 7):
+        s = abi.sambay_status_string(code)
+        assert s and s != "unknown status"
+    assert abi.sambay_status_string(99) == "unknown status"
+
+
+def test_workspace_queries(lib):
+    d = abi.make_dims(1, 2048, 2560, 5120, 16, 4, 160, abi.BF16)
+    T, Di, ldx, R = 2048, 5120, 192, 160
+    def r256(x):
+        return (x + 255) // 256 * 256
+    # uc as the bf16 split pair (4 bytes per element) + x_proj split-K partials
+    # (9 splits for 16 row tiles over 160 k-blocks; 16 splits for one row tile)
+    # + xdbl + split delta (bf16, 2 x dt_rank padded to 192) + dt (f32)
+    Rp = 192
+    want = (r256(T * Di * 4) + r256(9 * T * ldx * 4) + r256(T * ldx * 4) + r256(T * 2 * Rp * 2)
+            + r256(T * Di * 4))
+    assert abi.sambay_scan_prefill_workspace(d) == want
+    assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == \
+        r256(64 * Di * 4) + r256(16 * 64 * ldx * 4) + r256(64 * ldx * 4) + r256(64 * 2 * Rp * 2) \
+        + r256(64 * Di * 4)
+    # float32 mode: no partials, no split delta
+    f = abi.make_dims(1, 64, 64, 128, 16, 4, 4, abi.F32)
+    assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4)
+    assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2)
+    assert abi.gmu_step_workspace(d, 64) > 64 * 5120 * 2
+    # invalid or unsupported dims -> 0
+    assert abi.sambay_scan_prefill_workspace(abi.make_dims(1, 16, 64, 128, 8, 4, 8, abi.BF16)) == 0
+    assert abi.sambay_scan_prefill_workspace(abi.make_dims(0, 16, 64, 128)) == 0
+    assert abi.gmu_step_workspace(d, 257) == 0
+    assert abi.gmu_forward_workspace(abi.make_dims(1, 1, 100, 128), 4) == 0
+
+
+class _FakePtr:
+    """Stands in for a tensor in calls that must fail validation."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return 1
+
+    def element_size(self):
+        return 1
+
+
+def _weights(addr=0x10000):
+    return abi.ScanWeights(*([addr] * 7))
+
+
+def test_scan_argument_errors(lib):
+    d = abi.make_dims(1, 16, 64, 128, 16, 4, 8, abi.BF16)
+    p = _FakePtr(0x10000)
+    st = 0
+    # NULL input
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), d, None, p, p, p, True, p, st)
+    assert e.value.code == 1
+    # NULL weight pointer
+    w = _weights(); w.A = None
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(w, d, p, _FakePtr(0x20000), p, p, True, p, st)
+    assert e.value.code == 1
+    # misaligned pointer
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), d, _FakePtr(0x10008), _FakePtr(0x20000), p, p, True, p, st)
+    assert e.value.code == 2
+    # M aliasing u
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), d, p, p, p, p, True, p, st)
+    assert e.value.code == 1
+    # unsupported d_state / d_conv / dt_rank
+    for bad in (abi.make_dims(1, 16, 64, 128, 8, 4, 8, abi.BF16),
+                abi.make_dims(1, 16, 64, 128, 16, 3, 8, abi.BF16),
+                abi.make_dims(1, 16, 64, 128, 16, 4, 12, abi.BF16),
+                abi.make_dims(1, 16, 64, 96, 16, 4, 8, abi.BF16)):
+        with pytest.raises(abi.SambayError) as e:
+            abi.sambay_scan_prefill(_weights(), bad, p, _FakePtr(0x20000), p, p, True, p, st)
+        assert e.value.code == 2
+    # bad enum / sizes
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), abi.make_dims(1, 0, 64, 128), p, _FakePtr(0x20000), p, p, True, p, st)
+    assert e.value.code == 1
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), abi.make_dims(1, 16, 64, 128, io=7), p, _FakePtr(0x20000), p, p, True, p, st)
+    assert e.value.code == 1
+    # workspace too small (1 byte)
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_prefill(_weights(), d, p, _FakePtr(0x20000), p, p, True, p, st)
+    assert e.value.code == 3
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_step(_weights(), d, p, _FakePtr(0x20000), p, p, p, st)
+    assert e.value.code == 3
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_scan_step(_weights(), d, p, p, p, p, p, st)
+    assert e.value.code == 1
+
+
+def test_gmu_argument_errors(lib):
+    d = abi.make_dims(1, 1, 64, 128, io=abi.BF16)
+    X, M, W1, W2, Y = (_FakePtr(a) for a in (0x10000, 0x20000, 0x30000, 0x40000, 0x50000))
+    tiny_ws = _FakePtr(0x60000)
+    st = 0
+    for fn in (abi.gmu_forward, abi.gmu_step):
+        with pytest.raises(abi.SambayError) as e:
+            fn(d, 4, X, M, W1, W2, None, Y, tiny_ws, st)
+        assert e.value.code == 3
+        with pytest.raises(abi.SambayError) as e:
+            fn(d, 4, None, M, W1, W2, None, Y, tiny_ws, st)
+        assert e.value.code == 1
+        with pytest.raises(abi.SambayError) as e:
+            fn(d, 0, X, M, W1, W2, None, Y, tiny_ws, st)
+        assert e.value.code == 1
+        with pytest.raises(abi.SambayError) as e:   # Y aliases M
+            fn(d, 4, X, M, W1, W2, None, M, tiny_ws, st)
+        assert e.value.code == 1
+        with pytest.raises(abi.SambayError) as e:   # d_model not a multiple of 64 in bf16
+            fn(abi.make_dims(1, 1, 96, 128, io=abi.BF16), 4, X, M, W1, W2, None, Y, tiny_ws, st)
+        assert e.value.code == 2
+    with pytest.raises(abi.SambayError) as e:
+        abi.gmu_step(d, 300, X, M, W1, W2, None, Y, tiny_ws, st)
+    assert e.value.code in (2, 3)
+
+
+def test_device_status_null_out(lib):
+    assert lib.sambay_device_status(None, None) == 1
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle, and fails loudly without the library."""
+    pkg = os.path.join(ROOT, "gated_memory_sharing_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert not re.search(r"^\s*(import|from)\s+oracle", src, re.M), fn
+    with pytest.raises(RuntimeError):
+        abi._lib_backup = abi._lib
+        try:
+            abi._lib = None
+            abi.load("/nonexistent/libsambay.so")
+        finally:
+            abi._lib = abi._lib_backup
