@@ -35,6 +35,7 @@ EXPORTS = (
     "gmu_step_workspace",
     "sambay_scan_prefill",
     "sambay_scan_step",
+    "sambay_scan_step_noalloc",
     "gmu_forward",
     "gmu_step",
     "sambay_device_status",
@@ -96,6 +97,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gmu_step_workspace": (sz, [pd, i64]),
         "sambay_scan_prefill": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]),
         "sambay_scan_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp, sz, vp]),
+        "sambay_scan_step_noalloc": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp]),
         "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sambay_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
@@ -169,6 +171,20 @@ def sambay_scan_step(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv
     _check("sambay_scan_step", load().sambay_scan_step(
         ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state),
         _p(conv_state), _p(ws), ws_bytes, _stream(stream)))
+
+
+# Library-owned scratch size of sambay_scan_step_noalloc (bytes, per GPU).
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def sambay_scan_step_noalloc(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv_state,
+                             stream=None):
+    """sambay_scan_step without a workspace argument, for callers that cannot
+    allocate device memory: the library uses a fixed scratch array of its own
+    (shared by all calls on a device, so calls must not overlap on the GPU)."""
+    _check("sambay_scan_step_noalloc", load().sambay_scan_step_noalloc(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state),
+        _p(conv_state), _stream(stream)))
 
 
 def gmu_forward(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=None):

@@ -440,6 +440,17 @@ sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* 
 
 }  // namespace
 
+// Scratch of sambay_scan_step_noalloc: a fixed array compiled into the
+// library, for callers that cannot allocate device memory.  Host code must
+// not pass this symbol to a kernel directly (on the host it names a host-side
+// stand-in); its device address is looked up per device with
+// cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SAMBAY_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+}  // namespace
+
 // ====================================================================== C ABI
 
 extern "C" {
@@ -576,6 +587,33 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   else { SAMBAY_STEP_GEMMS(256) }
 #undef SAMBAY_STEP_GEMMS
   return SAMBAY_OK;
+}
+
+sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const sambay_dims* d,
+                                       const void* u_t, void* m_t, float* ssm_state,
+                                       void* conv_state, sambay_stream_t stream) {
+  if (!d) return SAMBAY_ERR_INVALID_ARG;
+  sambay_dims e = *d;
+  e.seqlen = 1;
+  SAMBAY_TRY(check_dims(&e, false, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u_t, m_t, ssm_state, conv_state}));
+  if (m_t == u_t) return SAMBAY_ERR_INVALID_ARG;
+  if (sambay_scan_step_workspace(&e) > SAMBAY_NOALLOC_SCRATCH_BYTES) return SAMBAY_ERR_UNSUPPORTED;
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  if (g_noalloc_ptr[dev] == nullptr) {
+    // once per device, with that device current
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return SAMBAY_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  if (e.io == SAMBAY_BF16)
+    return scan_step_impl<bf16>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
+  return scan_step_impl<float>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
 }
 
 sambay_status sambay_device_status(sambay_stream_t stream, int32_t* out_code) {

@@ -171,6 +171,38 @@ SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const v
                        void* ws, size_t ws_bytes, sambay_stream_t stream);
 
 /*
+ * sambay_scan_step_noalloc - sambay_scan_step for callers that cannot
+ * allocate device memory.  The paper has no counterpart; this is a property
+ * of the library, not of the method.
+ *
+ * Some callers have no way to provide the `ws` buffer: a decode loop inside
+ * a serving engine whose memory is planned up front and that forbids
+ * allocation on the per-token path, or a plugin host that hands the library
+ * only its input and output pointers.  This variant takes the same
+ * arguments as sambay_scan_step minus the workspace and computes the same
+ * result with the same kernels; its scratch is a fixed array compiled into
+ * the library (SAMBAY_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that
+ * loads the library until the process exits).  It allocates nothing.
+ *
+ *   - Sizes whose sambay_scan_step_workspace(dims) exceeds
+ *     SAMBAY_NOALLOC_SCRATCH_BYTES are rejected with SAMBAY_ERR_UNSUPPORTED
+ *     before any launch (8 MiB covers 64 sequences at d_inner 5120).
+ *   - The first call on each device looks up the array's device address on
+ *     that device (so that device must be current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; nothing in it needs to start at zero.  Calls that overlap on
+ *     the GPU (different streams, or host threads without ordering) race on
+ *     it and give wrong results: order them.
+ */
+#define SAMBAY_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+SAMBAY_API sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w,
+                                                  const sambay_dims* dims, const void* u_t,
+                                                  void* m_t, float* ssm_state, void* conv_state,
+                                                  sambay_stream_t stream);
+
+/*
  * sambay_device_status - synchronise `stream`, then read and clear the
  * current device's status word.  *out_code receives the sambay_status a
  * kernel recorded (SAMBAY_OK if none).  Returns SAMBAY_ERR_CUDA if the
