@@ -40,11 +40,28 @@ __device__ __forceinline__ float silu(float x) {
   return __fdividef(x, 1.0f + ex2_approx(-x * kLog2e));
 }
 
-// softplus(x) = log(1 + e^x).  Above 20 the correction log1p(e^-x) < 2.1e-9
-// relative, below float32 resolution of x, so x is returned there; otherwise
-// log1p of the exponential, with CUDA's own log1pf.
+// log2(x) on the special-function unit (PTX lg2.approx.f32).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// softplus(x) = log(1 + e^x) = max(x, 0) + log1p(y),  y = e^-|x| in (0, 1].
+// log1p(y): for y < 1/16 its Taylor series y - y^2/2 + y^3/3 - y^4/4 + y^5/5
+// (the first omitted term is below 2e-7 of the sum); otherwise
+// log2(1 + y) * ln 2 with 1 + y >= 1.0625, where the SFU's absolute error in
+// log2 is a few 1e-7 of the result.  No cut-over to x is needed: for large x,
+// y underflows towards 0 and the series returns y.
 __device__ __forceinline__ float softplus(float x) {
-  return x > 20.0f ? x : log1pf(ex2_approx(x * kLog2e));
+  const float y = ex2_approx(-fabsf(x) * kLog2e);
+  float l;
+  if (y < 0.0625f) {
+    l = y * fmaf(-y, fmaf(-y, fmaf(-y, fmaf(-y, 0.2f, 0.25f), 0.33333334f), 0.5f), 1.0f);
+  } else {
+    l = lg2_approx(1.0f + y) * kLn2;
+  }
+  return fmaxf(x, 0.0f) + l;
 }
 
 // Pack / unpack helpers for 16-byte vector access.

@@ -118,7 +118,7 @@ int split_count(long long out_tiles, long long k, int max_splits) {
   return static_cast<int>((k_blocks + per - 1) / per);
 }
 
-constexpr int kXprojMaxSplits = 16;
+constexpr int kXprojMaxSplits = 64;
 
 // bf16 mode: x_proj reduces over K = 2*Di (the split uc pair)
 int xproj_splits(long long rows, int d_inner) {
@@ -197,19 +197,26 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch row_bytes),
-// box {64 inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_outer) {
+// 2-D tensor [outer, inner] (inner contiguous, row pitch row_bytes) with a
+// box of {box_inner, box_outer} elements whose inner extent is 128 bytes,
+// 128-byte swizzle, zero fill out of bounds (loads) / clipping (stores).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dtype, uint64_t inner,
+              uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  return fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 operand map, box {64, box_outer}
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_outer) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, inner, outer, row_bytes, 64, box_outer);
 }
 
 // ------------------------------------------------------------ tensor-core GEMM launch
@@ -226,7 +233,7 @@ template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
 sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArgs g, int splits,
                      cudaStream_t st) {
   using namespace sambay::tc;
-  using C = Cfg<BN, A_MN, B_MN>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
   static bool attr_set[kMaxDevices] = {};
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS>;
   if (!attr_set[dev]) {
@@ -239,6 +246,25 @@ sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArg
   // A K-major: [M, K] -> box {64 k, 128 m};  MN-major: [K, M] -> box {64 m, 64 k}
   if (!make_map(&ta, a.ptr, a.cols, a.rows, a.cols * 2, A_MN ? 64 : BM)) return SAMBAY_ERR_CUDA;
   if (!make_map(&tb, b.ptr, b.cols, b.rows, b.cols * 2, B_MN ? 64 : BN)) return SAMBAY_ERR_CUDA;
+  // row-major epilogue through TMA when the output columns come in whole
+  // blocks: bf16 outputs in 64-column blocks (aux in 128 x 64 boxes, stores in
+  // 32 x 64 boxes per warp), f32 outputs in 32 x 32 boxes
+  CUtensorMap taux, tout;
+  std::memset(&taux, 0, sizeof(taux));
+  std::memset(&tout, 0, sizeof(tout));
+  g.tma_epi = 0;
+  if (C::kTmaEpi && g.ldo % 8 == 0) {
+    const bool f32 = KIND == sambay::tc::EPI_SOFTPLUS;
+    if (g.N % (f32 ? 32 : 64) == 0) {
+      const uint64_t eb = f32 ? 4 : 2;
+      bool okm = make_map(&tout, g.out, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          g.N, g.M, g.ldo * eb, f32 ? 32 : 64, 32);
+      if (okm && g.aux != nullptr && !f32)
+        okm = make_map(&taux, g.aux, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.N, g.M, g.ldo * 2, 64, BM);
+      if (!okm) return SAMBAY_ERR_CUDA;
+      g.tma_epi = 1;
+    }
+  }
   g.m_tiles = (g.M + BM - 1) / BM;
   g.n_tiles = (g.N + BN - 1) / BN;
   g.k_blocks = (g.K + BK - 1) / BK;
@@ -247,7 +273,7 @@ sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArg
   g.splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
   g.tiles = g.m_tiles * g.n_tiles * g.splits;
   const int grid = std::min(g.tiles, sms);
-  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, g);
+  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, taux, tout, g);
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
 
@@ -324,15 +350,22 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
     else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
     else SAMBAY_TRY((run_tc<256, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    sambay::scan::xdbl_reduce_kernel<<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
-        part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+    if (L.splits >= 16)
+      sambay::scan::xdbl_reduce_kernel<8><<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(
+          part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+    else
+      sambay::scan::xdbl_reduce_kernel<1><<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
+          part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
     // the A operand is padded with zeros to Rp, W_dt reads zeros past R
     auto gd = tc_args(static_cast<int>(rows), Di, 2 * Rp, dt, Di, nullptr, w->dt_bias);
     gd.b_k_wrap = Rp;
     const Operand a_d{delta, rows, 2LL * Rp}, b_wdt{w->dt_proj_w, Di, R};
-    SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
+    if (rows <= sambay::tc::BM)   // one row tile (decode): narrower tiles, more CTAs
+      SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
+    else
+      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
     SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>(
@@ -347,6 +380,22 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
   return SAMBAY_OK;
 }
 
+template <typename T, int SPT>
+sambay_status launch_scan(int dev, const sambay::scan::ScanParams<T>& p, cudaStream_t st) {
+  using Smem = sambay::scan::ScanSmem<T, SPT>;
+  auto kern = sambay::scan::selective_scan_kernel<T, SPT>;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(Smem))) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  dim3 grid(p.Di / Smem::CH, p.B);
+  kern<<<grid, sambay::scan::kScanThreads, sizeof(Smem), st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+}
+
 template <typename T>
 sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
                                 const sambay_dims* d, const void* u, void* M, float* ssm_state,
@@ -359,10 +408,11 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
                                   static_cast<const T*>(w->conv_w),
                                   static_cast<const T*>(w->conv_b), uc, d->batch, d->seqlen,
                                   d->d_inner, zero_init};
-    constexpr int VEC = 16 / sizeof(T);
+    constexpr int VEC = 8 / sizeof(T);
+    constexpr int TT = 8;
     const long long threads =
-        static_cast<long long>(d->batch) * ((d->seqlen + 15) / 16) * (d->d_inner / VEC);
-    sambay::scan::conv_silu_kernel<T, 16><<<grid_for(threads, 256, sms), 256, 0, st>>>(p);
+        static_cast<long long>(d->batch) * ((d->seqlen + TT - 1) / TT) * (d->d_inner / VEC);
+    sambay::scan::conv_silu_kernel<T, TT><<<grid_for(threads, 256, sms), 256, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
   SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st));
@@ -383,8 +433,12 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     p.R = d->dt_rank;
     p.ldx = d->dt_rank + 2 * d->d_state;
     p.zero_init = zero_init;
-    dim3 grid(d->d_inner / sambay::scan::kScanCh, d->batch);
-    sambay::scan::selective_scan_kernel<T><<<grid, 128, 0, st>>>(p);
+    // 4 states per thread when there are at least two warps per SM
+    // sub-partition with it (shared-memory traffic per exp is half that of 2
+    // states per thread); otherwise 2 states per thread, for twice the warps
+    const long long warps4 = static_cast<long long>(d->batch) * d->d_inner * 4 / 32;
+    if (warps4 >= 8LL * sms) SAMBAY_TRY((launch_scan<T, 4>(dev, p, st)));
+    else SAMBAY_TRY((launch_scan<T, 2>(dev, p, st)));
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
   return SAMBAY_OK;

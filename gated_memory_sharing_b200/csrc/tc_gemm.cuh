@@ -90,6 +90,24 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// shared -> global tile store (bulk group); out-of-range rows/columns are clipped
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// generic-proxy shared-memory writes become visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -195,79 +213,134 @@ struct GemmArgs {
   int* counters;      // split-K arrival counters per (m, n) tile, zero on entry
   int b_k_wrap;       // > 0: B's k coordinate wraps at this multiple of 64, so an A
                       // of [hi | lo] halves meets the same B twice (split-bf16 operand)
+  int tma_epi;        // row-major gate / residual / softplus epilogue through TMA
+                      // (aux tile in, output tile out); set by the host when the
+                      // output's columns come in whole 64 (bf16) / 32 (f32) blocks
 };
 
-// The final op on one element.  `o` is the output's linear index.
+// The final op on one element.  `o` is the output's linear index, `a` the aux
+// value at o (M for the gate, the residual or 0 for EPI_RESID).
 template <int KIND>
-__device__ __forceinline__ void epi_store_one(const GemmArgs& g, long long o, int n, float v) {
+__device__ __forceinline__ void epi_store_one(const GemmArgs& g, long long o, int n, float v, float a) {
   if (KIND == EPI_F32_PARTIAL) {
     reinterpret_cast<float*>(g.out)[o] = v;
   } else if (KIND == EPI_GATE) {
-    const float m = to_f32(reinterpret_cast<const bf16*>(g.aux)[o]);
-    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(silu(v) * m);
+    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(silu(v) * a);
   } else if (KIND == EPI_RESID) {
-    const float r = g.aux ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o]) : 0.0f;
-    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(v + r);
+    reinterpret_cast<bf16*>(g.out)[o] = __float2bfloat16_rn(v + a);
   } else {
     reinterpret_cast<float*>(g.out)[o] = softplus(v + g.vec[n]);
   }
 }
 
-// One thread's 32 accumulator values of row `m`, columns [n0, n0 + 32).
-// TRANS: the output is stored transposed, out[n * ldo + m] (swap-AB GEMV).
+// Per-warp staging buffer for the epilogue: 32 rows x (128 + 16 pad) bytes.
+// The row pitch keeps the per-thread 16-byte row accesses conflict-free.
+constexpr int kEpiPitchF32 = 144;   // 32 floats + pad
+constexpr int kEpiPitchB16 = 80;    // 32 bf16 + pad
+constexpr int kEpiWarpBytes = 32 * kEpiPitchF32;
+
+// One warp's 32 x 32 output block: thread `lane` holds the 32 accumulator
+// values of row m = row0 + lane, columns [n0, n0 + 32).  All 32 lanes call
+// this together.  A full block of a row-major output is staged through shared
+// memory so every global load / store instruction of the warp covers whole
+// row segments (8 rows x 64 B of bf16, 4 rows x 128 B of f32) instead of 32
+// scattered 16-byte pieces; the aux tile (M, residual) comes in the same way.
+// TRANS (swap-AB decode, out[n * ldo + m]) and ragged column edges go element
+// by element, which is already coalesced across the warp for TRANS.
 template <int KIND, bool TRANS>
-__device__ __forceinline__ void epi_chunk(const GemmArgs& g, int m, int n0, const float (&v)[32]) {
-  if (m >= g.M) return;
+__device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row0, int lane, int n0,
+                                          const float (&v)[32], uint8_t* stage) {
+  const int m = row0 + lane;
   if (!TRANS && n0 + 32 <= g.N && (g.ldo % 8) == 0) {
-    // vectorised row segment: 32 contiguous outputs
-    const long long base = static_cast<long long>(m) * g.ldo + n0;
-    if (KIND == EPI_F32_PARTIAL) {
-      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + base);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    } else if (KIND == EPI_SOFTPLUS) {
-      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + base);
+    if (KIND == EPI_F32_PARTIAL || KIND == EPI_SOFTPLUS) {
+      float4* mine = reinterpret_cast<float4*>(stage + lane * kEpiPitchF32);
       const float4* bias = reinterpret_cast<const float4*>(g.vec + n0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float4 b = bias[j];
-        float4 r;
-        r.x = softplus(v[4 * j + 0] + b.x);
-        r.y = softplus(v[4 * j + 1] + b.y);
-        r.z = softplus(v[4 * j + 2] + b.z);
-        r.w = softplus(v[4 * j + 3] + b.w);
-        dst[j] = r;
+        float4 r = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        if (KIND == EPI_SOFTPLUS) {
+          const float4 b = bias[j];
+          r.x = softplus(r.x + b.x);
+          r.y = softplus(r.y + b.y);
+          r.z = softplus(r.z + b.z);
+          r.w = softplus(r.w + b.w);
+        }
+        mine[j] = r;
       }
+      __syncwarp();
+      float* out = reinterpret_cast<float*>(g.out);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = i * 4 + (lane >> 3), seg = lane & 7;
+        if (row0 + r < g.M)
+          *reinterpret_cast<float4*>(out + static_cast<long long>(row0 + r) * g.ldo + n0 + seg * 4) =
+              *reinterpret_cast<const float4*>(stage + r * kEpiPitchF32 + seg * 16);
+      }
+      __syncwarp();
     } else {
-      const uint4* auxv = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(g.aux) + base);
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + base);
+      const bool has_aux = KIND == EPI_GATE || g.aux != nullptr;
+      const bf16* aux = reinterpret_cast<const bf16*>(g.aux);
+      Pack16 a[4];
+      if (has_aux) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 8 + (lane >> 2), seg = lane & 3;
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (row0 + r < g.M)
+            x = *reinterpret_cast<const uint4*>(aux + static_cast<long long>(row0 + r) * g.ldo + n0 + seg * 8);
+          *reinterpret_cast<uint4*>(stage + r * kEpiPitchB16 + seg * 16) = x;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[j].u = *reinterpret_cast<const uint4*>(stage + lane * kEpiPitchB16 + j * 16);
+        __syncwarp();
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        Pack16 a, r;
-        if (KIND == EPI_GATE || g.aux) a.u = auxv[j];
+        Pack16 r;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float x0 = v[8 * j + 2 * e], x1 = v[8 * j + 2 * e + 1];
-          float y0, y1;
+          float y0 = x0, y1 = x1;
           if (KIND == EPI_GATE) {
-            const float2 mm = __bfloat1622float2(a.h2[e]);
+            const float2 mm = __bfloat1622float2(a[j].h2[e]);
             y0 = silu(x0) * mm.x;
             y1 = silu(x1) * mm.y;
-          } else if (g.aux) {
-            const float2 rr = __bfloat1622float2(a.h2[e]);
+          } else if (has_aux) {
+            const float2 rr = __bfloat1622float2(a[j].h2[e]);
             y0 = x0 + rr.x;
             y1 = x1 + rr.y;
-          } else {
-            y0 = x0;
-            y1 = x1;
           }
           r.h2[e] = __floats2bfloat162_rn(y0, y1);
         }
-        dst[j] = r.u;
+        *reinterpret_cast<uint4*>(stage + lane * kEpiPitchB16 + j * 16) = r.u;
       }
+      __syncwarp();
+      bf16* out = reinterpret_cast<bf16*>(g.out);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = i * 8 + (lane >> 2), seg = lane & 3;
+        if (row0 + r < g.M)
+          *reinterpret_cast<uint4*>(out + static_cast<long long>(row0 + r) * g.ldo + n0 + seg * 8) =
+              *reinterpret_cast<const uint4*>(stage + r * kEpiPitchB16 + seg * 16);
+      }
+      __syncwarp();
     }
     return;
+  }
+  if (m >= g.M) return;
+  // element by element (transposed output, or a ragged edge): all aux loads are
+  // issued before any store so they overlap; an element's own load still
+  // precedes its store, which keeps Y == residual aliasing safe
+  float a[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int n = n0 + j;
+    const long long o = TRANS ? static_cast<long long>(n) * g.ldo + m
+                              : static_cast<long long>(m) * g.ldo + n;
+    a[j] = 0.0f;
+    if (n < g.N && (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr)))
+      a[j] = to_f32(reinterpret_cast<const bf16*>(g.aux)[o]);
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
@@ -275,24 +348,38 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int m, int n0, cons
     if (n < g.N) {
       const long long o = TRANS ? static_cast<long long>(n) * g.ldo + m
                                 : static_cast<long long>(m) * g.ldo + n;
-      epi_store_one<KIND>(g, o, n, v[j]);
+      epi_store_one<KIND>(g, o, n, v[j], a[j]);
     }
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, bool A_MN, bool B_MN>
+constexpr int kSlotBytes = 16384;             // one 128-row x 128-byte epilogue block
+constexpr int kMaxDynSmem = 232448;           // 227 KB per CTA on sm_100
+
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
 struct Cfg {
   static constexpr int kABytes = BM * BK * 2;   // 16 KB
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  // TMA epilogue: bf16 outputs keep one 128 x 64 block per 64 output columns
+  // (the whole tile's aux arrives ahead of the accumulator); f32 outputs
+  // double-buffer 128 x 32 blocks
+  static constexpr bool kTmaEpi = !TRANS && (KIND == EPI_GATE || KIND == EPI_RESID || KIND == EPI_SOFTPLUS);
+  static constexpr int kSlots = !kTmaEpi ? 0 : (KIND == EPI_SOFTPLUS ? 2 : BN / 64);
+  static constexpr int kEpiBytes = kTmaEpi ? kSlots * kSlotBytes + 1024 /*bias*/ : 4 * kEpiWarpBytes;
+  static constexpr int kFixed = 1024 /*align slack*/ + 512 /*barriers*/ + kEpiBytes;
+  static constexpr int kStagesFit = (kMaxDynSmem - kFixed) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
-  static constexpr size_t kSmem = 1024 /*align slack*/ + static_cast<size_t>(kStages) * kStageBytes + 256;
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static constexpr size_t kSmem = static_cast<size_t>(kFixed) + static_cast<size_t>(kStages) * kStageBytes;
+  static_assert(kStages >= 2, "shared memory budget");
+  static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
+  static_assert(kSlots * kSlotBytes >= (kTmaEpi ? 4 * kEpiWarpBytes : 0), "fallback staging fits the slots");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, whole 32-column epilogue chunks");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element atoms");
 };
 
@@ -314,22 +401,27 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmAux, const __grid_constant__ CUtensorMap tmOut,
                    const GemmArgs g) {
-  using C = Cfg<BN, A_MN, B_MN>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint8_t* epi_area = smem + S * C::kStageBytes;          // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_area + C::kEpiBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;      // [2]
   uint64_t* tempty = tfull + 2;     // [2]
   uint64_t* drain = tempty + 2;     // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* auxf = drain + 1;       // [4] aux block landed (TMA epilogue)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxf + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;
+  uint8_t* epi_stage = epi_area;                           // fallback staging, 4 x kEpiWarpBytes
+  float* epi_vec = reinterpret_cast<float*>(epi_area + C::kSlots * kSlotBytes);  // tile's bias
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -344,12 +436,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], 4);
     }
     mbar_init(drain, 1);
+    for (int j = 0; j < 4; ++j) mbar_init(&auxf[j], 1);
     *abort_flag = 0;
     *last_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (C::kTmaEpi && g.tma_epi) {
+      if (KIND != EPI_SOFTPLUS && g.aux != nullptr) prefetch_tmap(&tmAux);
+      prefetch_tmap(&tmOut);
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -447,20 +544,136 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ epilogue
     const int quarter = warp & 3;            // TMEM lanes [32*quarter, +32)
     const int ep_tid = threadIdx.x - 64;     // 0..127
+    uint8_t* my_stage = epi_stage + (warp - 2) * kEpiWarpBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t aux_phase = 0;    // parity bit per aux slot
+    const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     for (int t = blockIdx.x; t < g.tiles; t += gridDim.x) {
       const TileCoord c = tile_coord(g, t);
       const bool split = g.splits > 1 && KIND != EPI_F32_PARTIAL;
+      const bool tma = C::kTmaEpi && g.tma_epi && !split;
+      if (tma) {
+        // the tile's aux blocks (M or the residual) and bias are fetched while
+        // its main loop still runs; the slots are free because every store of
+        // the previous tile has finished reading them (barrier at tile end)
+        if (has_aux && ep_tid == 0) {
+#pragma unroll
+          for (int j = 0; j < C::kSlots; ++j) {
+            const int n0 = c.n * BN + 64 * j;
+            if (n0 < g.N) {
+              mbar_arrive_expect_tx(&auxf[j], kSlotBytes);
+              tma_load_2d(epi_area + j * kSlotBytes, &tmAux, &auxf[j], n0, c.m * BM);
+            }
+          }
+        }
+        if (KIND == EPI_SOFTPLUS)
+          for (int i = ep_tid; i < BN; i += 128)
+            epi_vec[i] = c.n * BN + i < g.N ? g.vec[c.n * BN + i] : 0.0f;
+      }
       bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
-      // the split-K path synchronises the 4 epilogue warps, so they must agree
-      // on leaving the loop together
-      if (split) ok = epi_agree(ok);
+      // the split-K and TMA paths synchronise the 4 epilogue warps, so they must
+      // agree on leaving the loop together (the barrier also publishes epi_vec)
+      if (split || tma) ok = epi_agree(ok);
       if (!ok) break;
       tc_fence_after();
       const int row = c.m * BM + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      if (tma) {
+        // rows r of the tile live at r * 128 bytes of a slot, 16-byte chunks
+        // 128-byte swizzled (the layout TMA reads and writes)
+        const int r = quarter * 32 + lane;
+        if (KIND == EPI_SOFTPLUS) {
+#pragma unroll 1
+          for (int ch = 0; ch < BN / 32; ++ch) {
+            const int n0 = c.n * BN + 32 * ch;
+            if (n0 >= g.N) break;
+            uint8_t* blk = epi_area + (ch & 1) * kSlotBytes;
+            if (ch >= 2) {            // this slot's store from two chunks ago has read it
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+            }
+            uint32_t rr[32];
+            tmem_ld_32x32b_x32(t_row + 32 * ch, rr);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 b = *reinterpret_cast<const float4*>(epi_vec + 32 * ch + 4 * k);
+              float4 o;
+              o.x = softplus(__uint_as_float(rr[4 * k + 0]) + b.x);
+              o.y = softplus(__uint_as_float(rr[4 * k + 1]) + b.y);
+              o.z = softplus(__uint_as_float(rr[4 * k + 2]) + b.z);
+              o.w = softplus(__uint_as_float(rr[4 * k + 3]) + b.w);
+              *reinterpret_cast<float4*>(blk + r * 128 + ((k ^ (r & 7)) << 4)) = o;
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, c.m * BM + quarter * 32);
+              bulk_commit();
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int j = 0; j < C::kSlots; ++j) {
+            const int n0 = c.n * BN + 64 * j;
+            if (n0 >= g.N) break;
+            uint8_t* blk = epi_area + j * kSlotBytes;
+            if (has_aux) {
+              ok = mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag);
+              ok = epi_agree(ok);
+              if (!ok) break;
+              aux_phase ^= 1u << j;
+            }
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+              uint32_t rr[32];
+              tmem_ld_32x32b_x32(t_row + 64 * j + 32 * h, rr);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const int k = 4 * h + kk;
+                uint4* addr = reinterpret_cast<uint4*>(blk + r * 128 + ((k ^ (r & 7)) << 4));
+                Pack16 a, o;
+                if (has_aux) a.u = *addr;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float x0 = __uint_as_float(rr[8 * kk + 2 * e]);
+                  const float x1 = __uint_as_float(rr[8 * kk + 2 * e + 1]);
+                  float y0 = x0, y1 = x1;
+                  if (KIND == EPI_GATE) {
+                    const float2 mm = __bfloat1622float2(a.h2[e]);
+                    y0 = silu(x0) * mm.x;
+                    y1 = silu(x1) * mm.y;
+                  } else if (has_aux) {
+                    const float2 rs = __bfloat1622float2(a.h2[e]);
+                    y0 = x0 + rs.x;
+                    y1 = x1 + rs.y;
+                  }
+                  o.h2[e] = __floats2bfloat162_rn(y0, y1);
+                }
+                *addr = o.u;
+              }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, c.m * BM + quarter * 32);
+              bulk_commit();
+            }
+          }
+          if (!ok) break;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        // every store of this tile has read its slot before the next tile's
+        // aux loads and bias overwrite them
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        continue;
+      }
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
         uint32_t r[32];
@@ -486,9 +699,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (KIND == EPI_F32_PARTIAL) {
           GemmArgs gs = g;
           gs.out = reinterpret_cast<float*>(g.out) + static_cast<long long>(c.split) * g.split_stride;
-          epi_chunk<KIND, TRANS>(gs, row, n0, v);
+          epi_chunk<KIND, TRANS>(gs, row - lane, lane, n0, v, my_stage);
         } else {
-          epi_chunk<KIND, TRANS>(g, row, n0, v);
+          epi_chunk<KIND, TRANS>(g, row - lane, lane, n0, v, my_stage);
         }
       }
       tc_fence_before();
@@ -511,26 +724,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (*last_flag) {
           __threadfence();
-          if (row < g.M) {
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-              const int n0 = c.n * BN + ch * 32;
-              float v[32];
+          for (int ch = 0; ch < BN / 32; ++ch) {
+            const int n0 = c.n * BN + ch * 32;
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            // split order is fixed; each split's 32 loads are in flight together
+#pragma unroll 1
+            for (int sp = 0; sp < g.splits; ++sp) {
+              const float* part = g.partials + static_cast<long long>(sp) * g.split_stride;
+              float x[32];
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 const int n = n0 + j;
-                v[j] = 0.0f;
-                if (n < g.N) {
-                  const long long o = TRANS ? static_cast<long long>(n) * g.ldo + row
-                                            : static_cast<long long>(row) * g.ldo + n;
-                  float acc = 0.0f;
-                  for (int sp = 0; sp < g.splits; ++sp)
-                    acc += __ldcg(g.partials + static_cast<long long>(sp) * g.split_stride + o);
-                  v[j] = acc;
-                }
+                const long long o = TRANS ? static_cast<long long>(n) * g.ldo + row
+                                          : static_cast<long long>(row) * g.ldo + n;
+                x[j] = (n < g.N && row < g.M) ? __ldcg(part + o) : 0.0f;
               }
-              epi_chunk<KIND, TRANS>(g, row, n0, v);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += x[j];
             }
+            epi_chunk<KIND, TRANS>(g, row - lane, lane, n0, v, my_stage);
           }
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -538,6 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (C::kTmaEpi && warp >= 2 && lane == 0) bulk_wait_read<0>();   // no store still reading smem
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -55,14 +55,15 @@ def test_workspace_queries(lib):
     def r256(x):
         return (x + 255) // 256 * 256
     # uc as the bf16 split pair (4 bytes per element) + x_proj split-K partials
-    # (9 splits for 16 row tiles over 160 k-blocks; 16 splits for one row tile)
+    # (9 splits for 16 row tiles over 160 k-blocks; 54 splits of 3 k-blocks for
+    # one row tile)
     # + xdbl + split delta (bf16, 2 x dt_rank padded to 192) + dt (f32)
     Rp = 192
     want = (r256(T * Di * 4) + r256(9 * T * ldx * 4) + r256(T * ldx * 4) + r256(T * 2 * Rp * 2)
             + r256(T * Di * 4))
     assert abi.sambay_scan_prefill_workspace(d) == want
     assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == \
-        r256(64 * Di * 4) + r256(16 * 64 * ldx * 4) + r256(64 * ldx * 4) + r256(64 * 2 * Rp * 2) \
+        r256(64 * Di * 4) + r256(54 * 64 * ldx * 4) + r256(64 * ldx * 4) + r256(64 * 2 * Rp * 2) \
         + r256(64 * Di * 4)
     # float32 mode: no partials, no split delta
     f = abi.make_dims(1, 64, 64, 128, 16, 4, 4, abi.F32)
