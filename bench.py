@@ -34,9 +34,16 @@ sys.path.insert(0, ROOT)
 from gated_memory_sharing_b200 import synth  # noqa: E402
 
 WORKLOAD = "prefill_b1_l2048"
+# DRAM bytes (read + write) per launch of a kernel, from one ncu capture of the
+# benchmarked workload (profiles/); None once the kernel has changed since.
+DRAM_TRAFFIC = {"selective_scan": 88.83e6}   # profiles/prefill_b1_l2048_launches.md
 METRIC = "scan+GMU prefill tokens/s"
 UNIT = "tokens/s"
-PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+# Special-function-unit exp2 rate per SM per clock (4 lanes per sub-partition
+# x 4 sub-partitions; checked on this B200 with an ex2.approx throughput probe)
+SFU_EX2_PER_SM_CLK = 16
 L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
 DECODE_BATCH = 64
 DECODE_RING = 64             # decode steps per captured graph
@@ -195,6 +202,31 @@ def run_reference(args, world, rank):
     }), flush=True)
 
 
+def kernel_work(name, d, sms, peaks, peak_kind):
+    """(bound, algorithmic units per launch, unit, peak) of one kernel of the
+    prefill step on dims d.  Algorithmic = what the method must compute or move
+    once: exps for the scan, 2*M*N*K flops for the GEMMs, bytes read + written
+    by the memory-bound kernels (inputs once, outputs once)."""
+    T, Di, Dm, N, R = d.tokens, d.d_inner, d.d_model, d.d_state, d.dt_rank
+    ldx, Rp = R + 2 * N, (R + 63) // 64 * 64
+    hbm = peaks["hbm_gbs"]
+    if name == "selective_scan":
+        peak = SFU_EX2_PER_SM_CLK * sms * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e9
+        return "alu", T * Di * N, "Gexp/s", peak, \
+            f"SFU ex2: {SFU_EX2_PER_SM_CLK}/SM/clk x {sms} SMs x max SM clock ({peak_kind} clock)"
+    if name in ("gmu_gate_gemm", "gmu_out_gemm"):
+        return "tensor", 2.0 * T * Dm * Di, "TFLOP/s", peaks["bf16_tflops"], f"{peak_kind} burst bf16"
+    if name == "conv_silu":      # u in (bf16), uc split pair out (2 x bf16)
+        return "hbm", T * Di * (2 + 4), "GB/s", hbm, f"{peak_kind} HBM copy"
+    if name == "x_proj":         # uc pair in, x_proj_w in, (delta|B|C) f32 out
+        return "hbm", T * Di * 4 + ldx * Di * 2 + T * ldx * 4, "GB/s", hbm, f"{peak_kind} HBM copy"
+    if name == "xdbl_reduce":    # (delta|B|C) out + split delta pair out; partials are scratch
+        return "hbm", T * ldx * 4 + T * 2 * Rp * 2, "GB/s", hbm, f"{peak_kind} HBM copy"
+    if name == "dt_proj":        # delta pair + W_dt in, dt f32 out
+        return "hbm", T * 2 * Rp * 2 + Di * R * 2 + T * Di * 4, "GB/s", hbm, f"{peak_kind} HBM copy"
+    return None
+
+
 def cpu_baseline_oracle(min_seconds=10.0, max_reps=4):
     """The oracle as it stands, on the full benchmark step, timed on this host."""
     from oracle import sambay_ref as ref
@@ -283,7 +315,24 @@ def run_ours(args, world, rank, local):
     step_ms = [a + b for a, b in zip(scan_ms, gmu_ms)]
     total_ms = max_over_ranks(sum(step_ms), world, device)
     value = world * args.steps * T / (total_ms / 1e3)
-    launches_per_step = 5 + 2   # conv, x_proj GEMM, x_proj reduce, dt_proj GEMM, scan; 2 GMU GEMMs
+
+    # ---- per-kernel timing: the same steps again, each of the library's
+    # launches bracketed by CUDA events on its stream
+    per_kernel = {}
+    launches_per_step = None
+    kt_steps = max(3, min(args.steps, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(kt_steps):
+        flush.fill_(float(i))
+        with abi.KernelTimer(max_launches=32) as kt:
+            step()
+            gmu_step()
+        torch.cuda.synchronize()
+        launches_per_step = len(kt.names)
+        for name, ms in kt.durations_ms():
+            per_kernel.setdefault(name, []).append(ms)
+    barrier(world)
 
     # ---- end to end through the ABI with host buffers
     u_host = u.cpu().pin_memory()
@@ -314,16 +363,29 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     assert abi.sambay_device_status() == 0
 
-    # ---- roofline of the dominant kernel pair (the GMU's two tcgen05 GEMMs)
-    gmu_mean_ms = statistics.mean(gmu_ms)
-    gmu_flops = 4.0 * T * Dm * Di
-    achieved_tf = gmu_flops / (gmu_mean_ms / 1e3) / 1e12
-    peak_tf = peaks["bf16_tflops"]
-    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_tf, "traffic": None,
-                "kernel": "gmu_forward: tc_gemm_kernel x2 (X W1^T + gate, H W2)",
-                "peak_kind": f"{peak_kind} burst bf16"}
+    # ---- roofline of every kernel; the dominant one (longest per step) leads
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    kernels = []
+    for name, ms_list in per_kernel.items():
+        launches = len(ms_list) / kt_steps
+        ms = statistics.mean(ms_list)
+        entry = {"kernel": name, "launches_per_step": launches, "ms": ms}
+        kw = kernel_work(name, d, sms, peaks, peak_kind)
+        if kw is not None:
+            bound, units, unit, peak, peak_note = kw
+            scale = 1e12 if unit == "TFLOP/s" else 1e9
+            achieved = units / (ms / 1e3) / scale
+            entry.update({"bound": bound, "algorithmic_per_launch": units, "achieved": achieved,
+                          "peak": peak, "unit": unit, "frac": achieved / peak, "peak_note": peak_note})
+        kernels.append(entry)
+    kernels.sort(key=lambda e: -e["ms"] * e["launches_per_step"])
+    dom = kernels[0]
+    roofline = {"bound": dom.get("bound"), "achieved": dom.get("achieved"), "peak": dom.get("peak"),
+                "unit": dom.get("unit"), "frac": dom.get("frac"),
+                "traffic": DRAM_TRAFFIC.get(dom["kernel"]), "kernel": dom["kernel"],
+                "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
     scan_mean_ms = statistics.mean(scan_ms)
+    gmu_mean_ms = statistics.mean(gmu_ms)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -335,10 +397,11 @@ def run_ours(args, world, rank, local):
                    "l2": "flushed between steps (256 MB write, outside the step events)"},
         "roofline": roofline,
         "breakdown_ms": {"scan_prefill": scan_mean_ms, "gmu_forward": gmu_mean_ms},
+        "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": u.numel() * 2 + X.numel() * 2,
                 "d2h_bytes_per_step": Y.numel() * 2},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps,   # counted by the library's launch hook
         "clocks": clk,
     }
     if decode is not None:
@@ -392,6 +455,17 @@ def bench_decode(args, scan, gmu, d, seed, flush, stream, world, device, peaks):
     barrier(world)
     total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
     step_us = 1e3 * total_ms / (reps * DECODE_RING)
+    # per-kernel breakdown of a few eager steps (launch gaps excluded)
+    from gated_memory_sharing_b200 import abi
+    per_kernel = {}
+    for i in range(4):
+        with abi.KernelTimer(max_launches=32) as kt:
+            scan.step(ring_u[i], h, cs, m_t=m)
+            gmu.step(ring_x[i], m, residual=True, Y=y[i])
+        torch.cuda.synchronize()
+        for name, ms in kt.durations_ms():
+            per_kernel.setdefault(name, []).append(1e3 * ms)
+    kernels_us = {k: statistics.mean(v) for k, v in per_kernel.items()}
     # algorithmic bytes per decode step (every byte the step must move once)
     state = B * Di * d.d_state * 4 * 2 + B * Di * d.d_conv * 2 * 2
     weights = (d.dt_rank + 2 * d.d_state) * Di * 2 + Di * d.dt_rank * 2 + Di * (d.d_conv + 1) * 2 \
@@ -406,6 +480,7 @@ def bench_decode(args, scan, gmu, d, seed, flush, stream, world, device, peaks):
             "setup": "16-token prompt prefill; the decode state has a fixed size, so the step "
                      "cost does not depend on the position",
             "l2": "flushed between graph replays of 64 back-to-back steps",
+            "kernels_us": kernels_us,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_step": nbytes}}

@@ -38,6 +38,8 @@ EXPORTS = (
     "sambay_scan_step_noalloc",
     "gmu_forward",
     "gmu_step",
+    "sambay_profile_begin",
+    "sambay_profile_end",
     "sambay_device_status",
     "sambay_status_string",
     "sambay_version",
@@ -100,6 +102,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sambay_scan_step_noalloc": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp]),
         "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sambay_profile_begin": (ctypes.c_int, [ctypes.POINTER(vp), i32]),
+        "sambay_profile_end": (i32, [ctypes.POINTER(ctypes.c_char_p), i32]),
         "sambay_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
         "sambay_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "sambay_version": (ctypes.c_char_p, []),
@@ -199,6 +203,38 @@ def gmu_step(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=None):
     _check("gmu_step", load().gmu_step(
         ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(residual), _p(Y), _p(ws),
         ws_bytes, _stream(stream)))
+
+
+class KernelTimer:
+    """Times each kernel the library launches, with caller-owned CUDA events.
+
+        with KernelTimer(max_launches=64) as kt:
+            ...library calls...
+        kt.durations_ms()   # [(kernel name, ms), ...] in launch order
+    """
+
+    def __init__(self, max_launches: int = 256):
+        import torch
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * max_launches)]
+        for e in self.events:          # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+        self.names = []
+
+    def __enter__(self):
+        _check("sambay_profile_begin", load().sambay_profile_begin(self._handles, len(self.events)))
+        return self
+
+    def __exit__(self, *exc):
+        buf = (ctypes.c_char_p * (len(self.events) // 2))()
+        n = load().sambay_profile_end(buf, len(buf))
+        self.names = [buf[i].decode() for i in range(n)]
+        return False
+
+    def durations_ms(self):
+        return [(name, self.events[2 * i].elapsed_time(self.events[2 * i + 1]))
+                for i, name in enumerate(self.names)]
 
 
 def sambay_device_status(stream=None) -> int:

@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "../../include/sambay.h"
 #include "common.cuh"
@@ -49,6 +50,39 @@ sambay_status current_device(int* dev_out, int* sms_out) {
   *sms_out = d.sms;
   return SAMBAY_OK;
 }
+
+// ------------------------------------------------------------ kernel timing
+//
+// While a measurement session is open on the calling thread
+// (sambay_profile_begin), every kernel launch records the caller's events
+// 2i and 2i+1 on its stream around the i-th launch and remembers the kernel's
+// name.  Host-side bookkeeping only; closed sessions cost one branch.
+
+struct ProfState {
+  cudaEvent_t* ev = nullptr;
+  int cap = 0;      // events available
+  int n = 0;        // events used
+  std::vector<const char*> names;
+};
+thread_local ProfState* g_prof = nullptr;
+thread_local ProfState g_prof_storage;
+
+struct ProfScope {
+  cudaStream_t st;
+  bool on;
+  ProfScope(const char* name, cudaStream_t s) : st(s), on(g_prof != nullptr && g_prof->n + 2 <= g_prof->cap) {
+    if (on) {
+      cudaEventRecord(g_prof->ev[g_prof->n], st);
+      g_prof->names.push_back(name);
+    }
+  }
+  ~ProfScope() {
+    if (on) {
+      cudaEventRecord(g_prof->ev[g_prof->n + 1], st);
+      g_prof->n += 2;
+    }
+  }
+};
 
 // ------------------------------------------------------------ validation
 
@@ -230,8 +264,8 @@ struct Operand {
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
 // split_count for the same sizes).
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
-sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArgs g, int splits,
-                     cudaStream_t st) {
+sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
+                     sambay::tc::GemmArgs g, int splits, cudaStream_t st) {
   using namespace sambay::tc;
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
   static bool attr_set[kMaxDevices] = {};
@@ -273,7 +307,10 @@ sambay_status run_tc(int dev, int sms, Operand a, Operand b, sambay::tc::GemmArg
   g.splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
   g.tiles = g.m_tiles * g.n_tiles * g.splits;
   const int grid = std::min(g.tiles, sms);
-  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, taux, tout, g);
+  {
+    ProfScope ps(name, st);
+    kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, taux, tout, g);
+  }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
 
@@ -297,8 +334,9 @@ sambay::tc::GemmArgs tc_args(int M, int N, int K, void* out, long long ldo, cons
 // ------------------------------------------------------------ fp32 GEMM launch
 
 template <int KIND>
-sambay_status run_simt(const sambay::simt::Args& g, cudaStream_t st) {
+sambay_status run_simt(const char* name, const sambay::simt::Args& g, cudaStream_t st) {
   dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
+  ProfScope ps(name, st);
   sambay::simt::simt_gemm_kernel<KIND><<<grid, 256, 0, st>>>(g);
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -346,16 +384,19 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     gx.b_k_wrap = Di;
     const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
     constexpr int P = sambay::tc::EPI_F32_PARTIAL;
-    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else SAMBAY_TRY((run_tc<256, false, false, P, false>(dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    if (L.splits >= 16)
-      sambay::scan::xdbl_reduce_kernel<8><<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(
-          part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
-    else
-      sambay::scan::xdbl_reduce_kernel<1><<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
-          part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    {
+      ProfScope ps_reduce("xdbl_reduce", st);
+      if (L.splits >= 16)
+        sambay::scan::xdbl_reduce_kernel<8><<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(
+            part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+      else
+        sambay::scan::xdbl_reduce_kernel<1><<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
+            part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+    }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
     // the A operand is padded with zeros to Rp, W_dt reads zeros past R
@@ -363,16 +404,16 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     gd.b_k_wrap = Rp;
     const Operand a_d{delta, rows, 2LL * Rp}, b_wdt{w->dt_proj_w, Di, R};
     if (rows <= sambay::tc::BM)   // one row tile (decode): narrower tiles, more CTAs
-      SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
+      SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
     else
-      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>(dev, sms, a_d, b_wdt, gd, 1, st)));
+      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
-    SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>(
+    SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
         simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
                   ldx, Di, xdbl, ldx),
         st));
-    SAMBAY_TRY(run_simt<sambay::simt::SOFTPLUS>(
+    SAMBAY_TRY(run_simt<sambay::simt::SOFTPLUS>("dt_proj_f32",
         simt_args(xdbl, ldx, 1, static_cast<const float*>(w->dt_proj_w), 1, R,
                   static_cast<int>(rows), Di, R, dt, Di, nullptr, w->dt_bias),
         st));
@@ -392,6 +433,7 @@ sambay_status launch_scan(int dev, const sambay::scan::ScanParams<T>& p, cudaStr
     attr_set[dev] = true;
   }
   dim3 grid(p.Di / Smem::CH, p.B);
+  ProfScope ps("selective_scan", st);
   kern<<<grid, sambay::scan::kScanThreads, sizeof(Smem), st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -412,6 +454,7 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     constexpr int TT = 8;
     const long long threads =
         static_cast<long long>(d->batch) * ((d->seqlen + TT - 1) / TT) * (d->d_inner / VEC);
+    ProfScope ps("conv_silu", st);
     sambay::scan::conv_silu_kernel<T, TT><<<grid_for(threads, 256, sms), 256, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
@@ -452,11 +495,15 @@ sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, con
   const ScanWs L = scan_ws_layout(d, B);
   T* uc = reinterpret_cast<T*>(ws + L.uc);
   constexpr int VEC = 16 / sizeof(T);
-  sambay::scan::step_conv_kernel<T><<<grid_for(B * (d->d_inner / VEC), 256, 1 << 20), 256, 0, st>>>(
+  {
+    ProfScope ps("step_conv", st);
+    sambay::scan::step_conv_kernel<T><<<grid_for(B * (d->d_inner / VEC), 256, 1 << 20), 256, 0, st>>>(
       static_cast<const T*>(u_t), static_cast<T*>(conv_state), static_cast<const T*>(w->conv_w),
       static_cast<const T*>(w->conv_b), uc, d->batch, d->d_inner);
+  }
   if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st));
+  ProfScope ps("step_scan", st);
   sambay::scan::step_scan_kernel<T><<<grid_for(B * d->d_inner * 4, 256, 1 << 20), 256, 0, st>>>(
       uc, reinterpret_cast<const float*>(ws + L.dt), reinterpret_cast<const float*>(ws + L.xdbl),
       w->A, w->D, ssm_state, static_cast<T*>(m_t), d->batch, d->d_inner, d->dt_rank,
@@ -471,11 +518,11 @@ sambay_status gmu_f32(const sambay_dims* d, long long rows, const void* X, const
                       const GmuWs& L, cudaStream_t st) {
   const int Dm = d->d_model, Di = d->d_inner;
   float* H = reinterpret_cast<float*>(ws + L.h);
-  SAMBAY_TRY(run_simt<sambay::simt::GATE>(
+  SAMBAY_TRY(run_simt<sambay::simt::GATE>("gmu_gate_f32",
       simt_args(static_cast<const float*>(X), Dm, 1, static_cast<const float*>(W1), 1, Dm,
                 static_cast<int>(rows), Di, Dm, H, Di, static_cast<const float*>(M)),
       st));
-  SAMBAY_TRY(run_simt<sambay::simt::RESID>(
+  SAMBAY_TRY(run_simt<sambay::simt::RESID>("gmu_out_f32",
       simt_args(H, Di, 1, static_cast<const float*>(W2), Dm, 1, static_cast<int>(rows), Dm, Di,
                 static_cast<float*>(Y), Dm, static_cast<const float*>(residual)),
       st));
@@ -601,10 +648,10 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false>(
-      dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st)));
+      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
   SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false>(
-      dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
+      "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st)));
   return SAMBAY_OK;
 }
@@ -633,8 +680,8 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   const auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual, nullptr, part, rows * static_cast<long long>(Dm), counters);
   const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
 #define SAMBAY_STEP_GEMMS(BNV)                                                                   \
-  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>(dev, sms, w1, xr, g1, L.splits1, st))); \
-  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>(dev, sms, w2, hr, g2, L.splits2, st)));
+  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, L.splits1, st))); \
+  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, L.splits2, st)));
   if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
   else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
   else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }
@@ -668,6 +715,25 @@ sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const samba
   if (e.io == SAMBAY_BF16)
     return scan_step_impl<bf16>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
   return scan_step_impl<float>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
+}
+
+sambay_status sambay_profile_begin(void* const* events, int32_t capacity) {
+  if (!events || capacity < 2) return SAMBAY_ERR_INVALID_ARG;
+  ProfState& ps = g_prof_storage;
+  ps.ev = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+  ps.cap = capacity & ~1;
+  ps.n = 0;
+  ps.names.clear();
+  g_prof = &ps;
+  return SAMBAY_OK;
+}
+
+int32_t sambay_profile_end(const char** names, int32_t max_names) {
+  if (!g_prof) return 0;
+  const int launches = g_prof->n / 2;
+  for (int i = 0; i < launches && names && i < max_names; ++i) names[i] = g_prof->names[i];
+  g_prof = nullptr;
+  return launches;
 }
 
 sambay_status sambay_device_status(sambay_stream_t stream, int32_t* out_code) {

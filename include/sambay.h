@@ -203,6 +203,20 @@ SAMBAY_API sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w,
                                                   sambay_stream_t stream);
 
 /*
+ * sambay_profile_begin / sambay_profile_end - per-kernel timing for
+ * measurement; the paper has no counterpart.  Between the two calls, on the
+ * calling thread, the i-th kernel the library launches is bracketed by
+ * cudaEventRecord(events[2i]) and cudaEventRecord(events[2i+1]) on its stream
+ * (events: caller-created cudaEvent_t handles, `capacity` of them; launches
+ * beyond capacity/2 are not recorded).  sambay_profile_end closes the session,
+ * writes up to max_names static kernel names (launch order) to `names` and
+ * returns the number of launches recorded.  Host bookkeeping only: nothing is
+ * synchronised or allocated on the device.
+ */
+SAMBAY_API sambay_status sambay_profile_begin(void* const* events, int32_t capacity);
+SAMBAY_API int32_t sambay_profile_end(const char** names, int32_t max_names);
+
+/*
  * sambay_device_status - synchronise `stream`, then read and clear the
  * current device's status word.  *out_code receives the sambay_status a
  * kernel recorded (SAMBAY_OK if none).  Returns SAMBAY_ERR_CUDA if the
