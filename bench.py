@@ -36,7 +36,9 @@ from gated_memory_sharing_b200 import synth  # noqa: E402
 WORKLOAD = "prefill_b1_l2048"
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture of the
 # benchmarked workload (profiles/); None once the kernel has changed since.
-DRAM_TRAFFIC = {"selective_scan": 88.83e6}   # profiles/prefill_b1_l2048_launches.md
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the current kernels,
+# from profiles/ (empty until captured again after a kernel change)
+DRAM_TRAFFIC = {}
 METRIC = "scan+GMU prefill tokens/s"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,

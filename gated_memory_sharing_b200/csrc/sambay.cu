@@ -163,7 +163,7 @@ int xproj_splits(long long rows, int d_inner) {
 int rank_pad(int R) { return (R + 63) / 64 * 64; }
 
 struct ScanWs {
-  size_t uc, part, xdbl, delta, dt, total;
+  size_t uc, part, xdbl, delta, dt, bcp, total;
   int splits;
 };
 
@@ -179,6 +179,8 @@ ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
   w.xdbl = off;  off += round256(static_cast<size_t>(T * ldx) * 4);
   w.delta = off; off += tc ? round256(static_cast<size_t>(T) * 2 * rank_pad(static_cast<int>(R)) * 2) : 0;
   w.dt = off;    off += round256(static_cast<size_t>(T * Di) * 4);
+  // B | C regrouped into token pairs: ceil(L / 2) pairs of 64 floats per sequence
+  w.bcp = off;   off += round256(static_cast<size_t>(d->batch) * ((T / d->batch + 1) / 2) * 64 * 4);
   w.total = off;
   return w;
 }
@@ -261,11 +263,33 @@ struct Operand {
   long long rows, cols;
 };
 
+// Last-wave balancing of a GEMM without K split: with W whole waves of
+// tiles over the SMs and a partial wave of `tail` tiles, the tail tiles are
+// cut along N into nsplit units (64 columns at the narrowest) so they spread
+// over up to all SMs instead of running on `tail` of them.
+struct TailPlan {
+  int full, nsplit;
+};
+
+TailPlan tail_plan(int tiles, int BN, int sms) {
+  TailPlan tp{tiles, 1};
+  const int waves = tiles / sms, tail = tiles % sms;
+  if (waves == 0 || tail == 0) return tp;
+  for (int cand = BN / 64; cand >= 2; cand /= 2)
+    if (BN % (cand * 64) == 0 && tail * cand <= sms) {
+      tp.full = waves * sms;
+      tp.nsplit = cand;
+      break;
+    }
+  return tp;
+}
+
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
-// split_count for the same sizes).
+// split_count for the same sizes); `balance_tail` (no K split) applies
+// tail_plan.
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
-                     sambay::tc::GemmArgs g, int splits, cudaStream_t st) {
+                     sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false) {
   using namespace sambay::tc;
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
   static bool attr_set[kMaxDevices] = {};
@@ -306,10 +330,22 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   g.kb_per_split = (g.k_blocks + splits - 1) / splits;
   g.splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
   g.tiles = g.m_tiles * g.n_tiles * g.splits;
+  g.full_tiles = g.tiles;
+  g.tail_nsplit = 1;
+  CUtensorMap tb2 = tb;
+  if (balance_tail && g.splits == 1) {
+    const TailPlan tp = tail_plan(g.tiles, BN, sms);
+    if (tp.nsplit > 1) {
+      if (!B_MN && !make_map(&tb2, b.ptr, b.cols, b.rows, b.cols * 2, BN / tp.nsplit)) return SAMBAY_ERR_CUDA;
+      g.tiles = tp.full + (g.tiles - tp.full) * tp.nsplit;
+      g.full_tiles = tp.full;
+      g.tail_nsplit = tp.nsplit;
+    }
+  }
   const int grid = std::min(g.tiles, sms);
   {
     ProfScope ps(name, st);
-    kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, taux, tout, g);
+    kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -372,6 +408,7 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
   const int Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
   float* xdbl = reinterpret_cast<float*>(ws + L.xdbl);
   float* dt = reinterpret_cast<float*>(ws + L.dt);
+  float* bcp = reinterpret_cast<float*>(ws + L.bcp);
   if (d->io == SAMBAY_BF16) {
     const bf16* uc = reinterpret_cast<const bf16*>(ws + L.uc);
     bf16* delta = reinterpret_cast<bf16*>(ws + L.delta);
@@ -392,10 +429,10 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
       ProfScope ps_reduce("xdbl_reduce", st);
       if (L.splits >= 16)
         sambay::scan::xdbl_reduce_kernel<8><<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(
-            part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+            part, L.splits, stride, xdbl, delta, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, Rp, ldx);
       else
         sambay::scan::xdbl_reduce_kernel<1><<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
-            part, L.splits, stride, xdbl, delta, static_cast<int>(rows), R, Rp, ldx);
+            part, L.splits, stride, xdbl, delta, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, Rp, ldx);
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
@@ -413,6 +450,12 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
         simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
                   ldx, Di, xdbl, ldx),
         st));
+    {
+      ProfScope ps_bc("bc_pairs", st);
+      sambay::scan::bc_pairs_kernel<<<grid_for(rows * 2 * d->d_state, 256, 1 << 20), 256, 0, st>>>(
+          xdbl, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, ldx);
+      if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+    }
     SAMBAY_TRY(run_simt<sambay::simt::SOFTPLUS>("dt_proj_f32",
         simt_args(xdbl, ldx, 1, static_cast<const float*>(w->dt_proj_w), 1, R,
                   static_cast<int>(rows), Di, R, dt, Di, nullptr, w->dt_bias),
@@ -421,20 +464,43 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
   return SAMBAY_OK;
 }
 
-template <typename T, int SPT>
-sambay_status launch_scan(int dev, const sambay::scan::ScanParams<T>& p, cudaStream_t st) {
-  using Smem = sambay::scan::ScanSmem<T, SPT>;
-  auto kern = sambay::scan::selective_scan_kernel<T, SPT>;
+// Channel runs of the prefill scan: CTAs per sequence (nblk) chosen so the
+// busiest SM carries the fewest channels, i.e. minimising
+// ceil(B * nblk / sms) * ceil(quads / nblk) over runs of at most kScanMaxCH
+// channels (ties: fewer, larger CTAs).  The split changes only which CTA
+// computes a channel, never its arithmetic.
+template <typename T>
+void scan_partition(sambay::scan::ScanParams<T>& p, int sms) {
+  using namespace sambay::scan;
+  const long long quads = p.Di / 4;
+  const long long lo = (quads + kScanMaxCH / 4 - 1) / (kScanMaxCH / 4);
+  long long best = lo, best_cost = -1;
+  for (long long nblk = lo; nblk <= quads; ++nblk) {
+    const long long cost = ((static_cast<long long>(p.B) * nblk + sms - 1) / sms) * ((quads + nblk - 1) / nblk);
+    if (best_cost < 0 || cost < best_cost) { best = nblk; best_cost = cost; }
+  }
+  p.nblk = static_cast<int>(best);
+  p.q_base = static_cast<int>(quads / best);
+  p.q_extra = static_cast<int>(quads % best);
+  p.chp = 4 * (p.q_base + (p.q_extra ? 1 : 0));
+}
+
+template <typename T>
+sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cudaStream_t st) {
+  using namespace sambay::scan;
+  auto kern = selective_scan_kernel<T>;
   static bool attr_set[kMaxDevices] = {};
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(Smem))) != cudaSuccess)
+                             ScanLayout(kScanMaxCH, sizeof(T)).bytes) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
     attr_set[dev] = true;
   }
-  dim3 grid(p.Di / Smem::CH, p.B);
+  scan_partition<T>(p, sms);
+  const ScanLayout ly(p.chp, sizeof(T));
+  dim3 grid(p.nblk, p.B);
   ProfScope ps("selective_scan", st);
-  kern<<<grid, sambay::scan::kScanThreads, sizeof(Smem), st>>>(p);
+  kern<<<grid, 8 * p.chp, ly.bytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
 
@@ -463,7 +529,7 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     sambay::scan::ScanParams<T> p{};
     p.uc = uc;
     p.dt = reinterpret_cast<const float*>(ws + L.dt);
-    p.xdbl = reinterpret_cast<const float*>(ws + L.xdbl);
+    p.bcp = reinterpret_cast<const float*>(ws + L.bcp);
     p.A = w->A;
     p.D = w->D;
     p.u = static_cast<const T*>(u);
@@ -473,15 +539,8 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     p.B = d->batch;
     p.L = d->seqlen;
     p.Di = d->d_inner;
-    p.R = d->dt_rank;
-    p.ldx = d->dt_rank + 2 * d->d_state;
     p.zero_init = zero_init;
-    // 4 states per thread when there are at least two warps per SM
-    // sub-partition with it (shared-memory traffic per exp is half that of 2
-    // states per thread); otherwise 2 states per thread, for twice the warps
-    const long long warps4 = static_cast<long long>(d->batch) * d->d_inner * 4 / 32;
-    if (warps4 >= 8LL * sms) SAMBAY_TRY((launch_scan<T, 4>(dev, p, st)));
-    else SAMBAY_TRY((launch_scan<T, 2>(dev, p, st)));
+    SAMBAY_TRY(launch_scan<T>(dev, sms, p, st));
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
   return SAMBAY_OK;
@@ -648,11 +707,11 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false>(
-      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st)));
+      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
   SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
-      st)));
+      st, true)));
   return SAMBAY_OK;
 }
 

@@ -31,6 +31,15 @@ namespace scan {
 constexpr int kN = 16;   // d_state
 constexpr int kK = 4;    // d_conv
 
+// B and C of each token pair, as the scan reads them: float index of B (which
+// = 0) or C (which = 1) of state n at token t of sequence b, Lh = ceil(L / 2)
+// pairs per sequence:
+//   [b * Lh + t / 2][which][n / 2][(t, n even), (t+1, n even), (t, n odd), (t+1, n odd)]
+__host__ __device__ inline long long bc_pair_index(int b, int t, int which, int n, int Lh) {
+  return (static_cast<long long>(b) * Lh + (t >> 1)) * 64 + which * 32 + (n >> 1) * 4 + (n & 1) * 2 + (t & 1);
+}
+
+
 // ---------------------------------------------------------------- cp.async
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
@@ -160,7 +169,8 @@ __global__ void __launch_bounds__(256) conv_silu_kernel(const ConvParams<T> p) {
 template <int LPG>
 __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int splits,
                                    long long split_stride, float* __restrict__ xdbl,
-                                   bf16* __restrict__ delta2, int rows, int R, int Rp, int ldx) {
+                                   bf16* __restrict__ delta2, float* __restrict__ bcp, int L,
+                                   int rows, int R, int Rp, int ldx) {
   const long long total4 = static_cast<long long>(rows) * ldx / 4;
   const int lane = threadIdx.x & 31, sub = lane % LPG;
   const long long warps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
@@ -203,6 +213,17 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
       reinterpret_cast<__nv_bfloat162*>(dh)[1] = __halves2bfloat162(hi[2], hi[3]);
       reinterpret_cast<__nv_bfloat162*>(dl)[0] = __halves2bfloat162(lo[0], lo[1]);
       reinterpret_cast<__nv_bfloat162*>(dl)[1] = __halves2bfloat162(lo[2], lo[3]);
+    } else {
+      // B | C columns, also regrouped into token pairs for the prefill scan
+      const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+      const int rr = static_cast<int>(row), b = rr / L, t = rr % L, Lh = (L + 1) >> 1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int cc = col + j - R;
+        const long long k = bc_pair_index(b, t, cc / kN, cc % kN, Lh);
+        bcp[k] = a[j];
+        if ((L & 1) && t == L - 1) bcp[k + 1] = 0.0f;   // the missing second token of the last pair
+      }
     }
   }
   // zero padding columns [R, Rp) of both halves
@@ -218,43 +239,67 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
   }
 }
 
+// B | C columns of xdbl regrouped into token pairs (bc_pair_index), for the
+// float32 path whose x_proj writes xdbl directly.  Thread: one (row, column).
+__global__ void bc_pairs_kernel(const float* __restrict__ xdbl, float* __restrict__ bcp, int L, int rows,
+                                int R, int ldx) {
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= static_cast<long long>(rows) * 2 * kN) return;
+  const int row = static_cast<int>(i / (2 * kN)), cc = static_cast<int>(i % (2 * kN));
+  const int b = row / L, t = row % L, Lh = (L + 1) >> 1;
+  const long long k = bc_pair_index(b, t, cc / kN, cc % kN, Lh);
+  bcp[k] = xdbl[static_cast<long long>(row) * ldx + R + cc];
+  if ((L & 1) && t == L - 1) bcp[k + 1] = 0.0f;
+}
+
 // ------------------------------------------------------- selective scan (prefill)
 //
-// CTA = CH channels of one sequence, 128 threads: thread (channel cl, lane q
-// of LANES = 16 / SPT) owns states q*SPT .. q*SPT + SPT-1 of channel cl, in
-// registers, for the whole sequence.  Tokens stream through shared memory in
-// chunks of TC, double buffered with cp.async; each lane's B and C values of
-// a token land side by side so one vector load fetches them.  Per chunk:
-//   prepass  (dt, dt*uc) and D*uc per (token, channel), once instead of once
-//     per lane;
-//   groups of 8 tokens: phase 1 issues every exp(dt A) and dt*uc*B of the
-//     group (independent of the state, so they overlap on the SFU), phase 2
-//     runs the dependent recurrence and this lane's share of each readout;
-//     a LANES-lane butterfly reduce-scatter then leaves lane q with the full
-//     readout of token (group base + q), which adds D*uc;
-//   the chunk's M rows leave with coalesced 16-byte stores.
-// Every shared-memory access is one wavefront of an SM-wide pipe, against
-// SPT exps per lane on the per-sub-partition SFU: SPT = 4 keeps the shared
-// memory pipe below the SFU.
+// Lane (channel c, quad q) of the 8 lanes of a channel owns states 2q, 2q+1
+// of c in registers for the whole sequence.  Costs that set the design, per
+// SM and clock on B200: 16 exp2 on the SFUs (one warp instruction holds an
+// SFU pipe for 8 clocks whatever its active mask), one shared-memory
+// wavefront (32 lanes x 32 bits: a 16-byte load per lane is 4 wavefronts),
+// and several warp shuffles.  Per token the 8 lanes of a channel need B and C
+// of their states (4 words each: shared memory), and dt, dt*uc of the channel
+// (2 words all 8 lanes share: one lane loads them for 8 tokens at a time and
+// shuffles hand them out), so shared memory stays below the SFUs.
+//
+// CTAs are sized per SM: a sequence's channels are cut into ScanParams::nblk
+// runs of 4-channel quads (q_base or q_base + 1 each), so at batch 1 one CTA
+// per SM holds 32 or 36 of the 5120 channels (8 or 9 warps).  Tokens stream
+// through shared memory in chunks of kScanTC, three in flight (cp.async): dt
+// and uc rows of the CTA's channels, and B, C as the x_proj reduction
+// regrouped them (bc_pair_index): one 16-byte load returns (B_t, B_t+1) of
+// states 2q and 2q+1, and likewise C.  Each thread's copies (one 4-element
+// piece of a dt, uc and output row) are fixed for the whole sequence, so the
+// chunk loop does no index arithmetic beyond a pointer step.  Token pairs run on the paired fp32 units (mul/fma .f32x2).
+// The readout sum over the 16 states is an 8-lane butterfly reduce-scatter
+// per 8 tokens, after which lane q holds token (base + q); it adds D*uc,
+// which the same lane preloaded, and the chunk's rows leave from a staging
+// tile.  One CTA barrier per chunk.
 
 template <typename T>
 struct ScanParams {
   const T* uc;          // [B*L, Di] (f32) or split pair [B*L, 2*Di] (bf16)
   const float* dt;      // [B*L, Di]
-  const float* xdbl;    // [B*L, ldx]: B at column R, C at column R + N
+  const float* bcp;     // [B * Lh * 64]: B and C per token pair (bc_pair_index)
   const float* A;       // [Di, N]
   const float* D;       // [Di]
   const T* u;           // [B, L, Di] raw scan input (for the new conv state)
   float* h;             // [B, Di, N] in/out
   T* conv_state;        // [B, Di, K] in/out
   T* M;                 // [B, L, Di] out
-  int B, L, Di, R, ldx;
+  int B, L, Di;
   int zero_init;
+  int nblk;             // CTAs per sequence (gridDim.x)
+  int q_base, q_extra;  // CTA i covers q_base (+1 if i < q_extra) quads of 4 channels
+  int chp;              // most channels of any CTA
 };
 
-constexpr int kScanThreads = 128;
 constexpr int kScanTC = 32;     // tokens per chunk
-constexpr int kScanPG = 8;      // tokens per pipeline group
+constexpr int kScanStages = 3;  // chunks in flight
+constexpr int kScanMaxCH = 36;  // channels per CTA at most (9 warps)
+constexpr int kScanMaxThreads = 8 * kScanMaxCH;
 
 // number of uc parts per element: the bf16 split pair (hi, lo) or one f32
 template <typename T>
@@ -263,202 +308,248 @@ __host__ __device__ constexpr int uc_parts() { return sizeof(T) == 2 ? 2 : 1; }
 template <typename T>
 __device__ __forceinline__ long long uc_ld(int Di) { return static_cast<long long>(Di) * uc_parts<T>(); }
 
-template <typename T, int SPT>
-struct ScanSmem {
-  static constexpr int LANES = kN / SPT;
-  static constexpr int CH = kScanThreads / LANES;
-  float dt[2][kScanTC][CH];
-  T uc[2][uc_parts<T>()][kScanTC][CH];
-  float bcq[2][kScanTC][LANES][2 * SPT];   // lane q: B[q*SPT ..], then C[q*SPT ..]
-  float2 dtdu[kScanTC][CH];                // (dt, dt * uc) of the current chunk
-  // rows padded: in the readout the lanes of a channel touch different tokens,
-  // and unpadded 128-byte rows would put them all on one bank
-  float dx[kScanTC][CH + 8];               // D * uc of the current chunk
-  T out[kScanTC][CH + 16 / sizeof(T)];
+// Dynamic shared memory of one CTA.  Rows of the channel tiles are `pitch`
+// elements, pitch = 4 (mod 32): a warp's 8-token x 4-channel preload then
+// touches 32 distinct banks.
+struct ScanLayout {
+  int pitch, dt, uc, bc, out, bytes;
+  __host__ __device__ ScanLayout(int chp, int tsize) {
+    pitch = chp + (36 - chp % 32) % 32;
+    const int parts = tsize == 2 ? 2 : 1;
+    dt = 0;
+    uc = dt + kScanStages * kScanTC * pitch * 4;
+    bc = uc + kScanStages * parts * kScanTC * pitch * tsize;
+    bc = (bc + 15) & ~15;
+    out = bc + kScanStages * kScanTC * 2 * kN * 4;
+    bytes = out + 2 * kScanTC * pitch * tsize;
+  }
 };
 
-template <typename T, int SPT>
-__device__ __forceinline__ float uc_value(const ScanSmem<T, SPT>& s, int buf, int t, int cl) {
-  if constexpr (sizeof(T) == 2) return to_f32(s.uc[buf][0][t][cl]) + to_f32(s.uc[buf][1][t][cl]);
-  else return s.uc[buf][0][t][cl];
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem_src) : "memory");
 }
-
 __device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(gmem_src) : "memory");
 }
 
-template <typename T, int SPT>
-__device__ __forceinline__ void scan_load_chunk(const ScanParams<T>& p, ScanSmem<T, SPT>& s, int buf,
-                                                int b, int c0, int t0, int nt) {
-  constexpr int CH = ScanSmem<T, SPT>::CH;
-  constexpr int LANES = ScanSmem<T, SPT>::LANES;
-  const int tid = threadIdx.x;
-  const long long row0 = static_cast<long long>(b) * p.L + t0;
-  constexpr int DTP = CH * 4 / 16;           // 16-byte pieces of a dt row
-  for (int i = tid; i < kScanTC * DTP; i += kScanThreads) {
-    const int t = i / DTP, piece = i % DTP;
-    float* d = &s.dt[buf][t][piece * 4];
-    if (t < nt) cp_async16(d, p.dt + (row0 + t) * p.Di + c0 + piece * 4);
-    else *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);  // dt = 0: h unchanged
-  }
-  // B and C of each lane's SPT states: two SPT-float pieces per (token, lane)
-  for (int i = tid; i < kScanTC * LANES * 2; i += kScanThreads) {
-    const int t = i / (LANES * 2), r = i % (LANES * 2);
-    const int q = r >> 1, which = r & 1;     // which: 0 = B, 1 = C
-    float* d = &s.bcq[buf][t][q][which * SPT];
-    const float* src = p.xdbl + (row0 + t) * p.ldx + p.R + which * kN + q * SPT;
-    if (t < nt) {
-      if constexpr (SPT == 4) cp_async16(d, src);
-      else cp_async8(d, src);
-    } else {
+// Paired fp32 arithmetic: two independent round-to-nearest operations.
+__device__ __forceinline__ unsigned long long f2_pack(float2 a) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_pack(a)), "l"(f2_pack(b)), "l"(f2_pack(c)));
+  return f2_unpack(r);
+}
+
+// One thread's share of every chunk's copies: a 4-element piece (row td,
+// columns 4 pd ..) of the dt row, of each uc part row and of the output row,
+// and 16-byte pieces of the chunk's B/C pairs.
+struct ScanPiece {
+  bool live;          // tid < 8 * CH: this thread owns a row piece
+  int soff;           // element offset of the piece within a stage's row tile
+  long long goff;     // element offset of the piece's token-0 position, [B*L, Di] layout
+  long long uoff;     // the same in the uc layout [B*L, parts * Di]
+};
+
+// Chunk loads.  Tokens past the end read as zeros: dt = 0 leaves h
+// unchanged and adds nothing.
+template <typename T>
+__device__ __forceinline__ void scan_load_chunk(const ScanParams<T>& p, uint8_t* smem, const ScanLayout& ly,
+                                                const ScanPiece& pc, int td, int st, int b, int t0) {
+  const int pitch = ly.pitch;
+  if (pc.live) {
+    const bool in = t0 + td < p.L;
+    const long long g = pc.goff + static_cast<long long>(t0) * p.Di;
+    float* d = reinterpret_cast<float*>(smem + ly.dt) + st * kScanTC * pitch + pc.soff;
+    if (in) cp_async16(d, p.dt + g);
+    else *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int NP = uc_parts<T>();
+    T* u = reinterpret_cast<T*>(smem + ly.uc) + st * NP * kScanTC * pitch + pc.soff;
+    const long long gu = pc.uoff + static_cast<long long>(t0) * NP * p.Di;
 #pragma unroll
-      for (int j = 0; j < SPT; ++j) d[j] = 0.0f;
+    for (int part = 0; part < NP; ++part) {
+      T* dp = u + part * kScanTC * pitch;
+      const T* src = p.uc + gu + part * p.Di;
+      if constexpr (sizeof(T) == 2) {
+        if (in) cp_async8(dp, src);
+        else *reinterpret_cast<uint2*>(dp) = make_uint2(0u, 0u);
+      } else {
+        if (in) cp_async16(dp, src);
+        else *reinterpret_cast<float4*>(dp) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
-  constexpr int UP = CH * sizeof(T) / 16;    // 16-byte pieces of a uc row part
-  constexpr int NP = uc_parts<T>();
-  for (int i = tid; i < kScanTC * UP * NP; i += kScanThreads) {
-    const int part = i / (kScanTC * UP);
-    const int r = i % (kScanTC * UP);
-    const int t = r / UP, piece = r % UP;
-    T* d = &s.uc[buf][part][t][piece * (16 / sizeof(T))];
-    if (t < nt)
-      cp_async16(d, p.uc + (row0 + t) * uc_ld<T>(p.Di) + part * p.Di + c0 + piece * (16 / sizeof(T)));
-    else
-      *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+  // B/C: the chunk's kScanTC / 2 pairs are 64 floats each, contiguous
+  const int Lh = (p.L + 1) >> 1;
+  const int pr0 = t0 >> 1;
+  float* s_bc = reinterpret_cast<float*>(smem + ly.bc) + st * kScanTC * 32;
+  const float* g_bc = p.bcp + (static_cast<long long>(b) * Lh + pr0) * 64;
+  for (int i = threadIdx.x; i < kScanTC * 8; i += blockDim.x) {
+    float* d = s_bc + 4 * i;
+    if (pr0 + (i >> 4) < Lh) cp_async16(d, g_bc + 4 * i);
+    else *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
-// Butterfly reduce-scatter over the LANES lanes of a channel: on entry v[i]
-// is this lane's partial for token i of the group; on return v[0] is the sum
-// over all lanes for token q (this lane's index among the LANES).
-template <int LANES>
-__device__ __forceinline__ float reduce_scatter(float (&v)[LANES], int q) {
+// Butterfly reduce-scatter over the 8 lanes of a channel (lanes 4q + c, q =
+// 0..7): on entry v[i] is this lane's partial for token i of the group; on
+// return the sum over the 8 lanes for token q.
+__device__ __forceinline__ float reduce_scatter8(float (&v)[8], int q) {
 #pragma unroll
-  for (int off = LANES / 2; off >= 1; off >>= 1) {
+  for (int off = 4; off >= 1; off >>= 1) {
     const bool upper = (q & off) != 0;
+    float keep[4], got[4];
 #pragma unroll
     for (int i = 0; i < off; ++i) {
       const float send = upper ? v[i] : v[i + off];
-      const float keep = upper ? v[i + off] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      keep[i] = upper ? v[i + off] : v[i];
+      got[i] = __shfl_xor_sync(0xffffffffu, send, off << 2);
+    }
+    if (off >= 2) {
+#pragma unroll
+      for (int i = 0; i < off; i += 2) {
+        const float2 r = add2(make_float2(keep[i], keep[i + 1]), make_float2(got[i], got[i + 1]));
+        v[i] = r.x;
+        v[i + 1] = r.y;
+      }
+    } else {
+      v[0] = keep[0] + got[0];
     }
   }
   return v[0];
 }
 
-template <typename T, int SPT>
-__global__ void __launch_bounds__(kScanThreads) selective_scan_kernel(const ScanParams<T> p) {
-  using Smem = ScanSmem<T, SPT>;
-  constexpr int LANES = Smem::LANES;
-  constexpr int CH = Smem::CH;
+// the chunk's readout rows from staging to M: this thread's 4-element piece
+template <typename T>
+__device__ __forceinline__ void scan_write_piece(const ScanParams<T>& p, const T* s_out, const ScanPiece& pc,
+                                                 int td, int t0, int nt) {
+  if (!pc.live || td >= nt) return;
+  T* dst = p.M + pc.goff + static_cast<long long>(t0) * p.Di;
+  if constexpr (sizeof(T) == 2) *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(s_out + pc.soff);
+  else *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(s_out + pc.soff);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(const ScanParams<T> p) {
   extern __shared__ __align__(16) uint8_t scan_smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>(scan_smem_raw);
-  const int cl = threadIdx.x / LANES;
-  const int q = threadIdx.x % LANES;
-  const int c0 = blockIdx.x * CH;
-  const int c = c0 + cl;
-  const int b = blockIdx.y;
-
-  float a2[SPT], h[SPT];
-#pragma unroll
-  for (int j = 0; j < SPT; ++j) {
-    a2[j] = p.A[c * kN + q * SPT + j] * kLog2e;
-    h[j] = p.zero_init ? 0.0f : p.h[(static_cast<long long>(b) * p.Di + c) * kN + q * SPT + j];
-  }
+  uint8_t* smem = scan_smem_raw;
+  const ScanLayout ly(p.chp, sizeof(T));
+  const int pitch = ly.pitch;
+  const int blk = blockIdx.x, b = blockIdx.y;
+  const int CH = 4 * (p.q_base + (blk < p.q_extra ? 1 : 0));
+  const int c0 = 4 * (blk * p.q_base + min(blk, p.q_extra));
+  // warp w: channels 4w .. 4w+3; lane 4q + c: states 2q, 2q+1 of channel 4w + c.
+  // State-major lanes: a half-warp's B/C loads touch 4 distinct 16-byte words.
+  const int lane = threadIdx.x & 31;
+  const int cl = (threadIdx.x >> 5) * 4 + (lane & 3), q = lane >> 2;
+  const bool active = cl < CH;
+  const int col = active ? cl : 0;               // lanes past CH shadow channel 0
+  const int c = c0 + col;
+  const float a2_0 = p.A[static_cast<long long>(c) * kN + 2 * q] * kLog2e;
+  const float a2_1 = p.A[static_cast<long long>(c) * kN + 2 * q + 1] * kLog2e;
+  float* hp = p.h + (static_cast<long long>(b) * p.Di + c) * kN + 2 * q;
+  float h0 = p.zero_init ? 0.0f : hp[0];
+  float h1 = p.zero_init ? 0.0f : hp[1];
+  const float Dc = p.D[c];
+  const float* s_dt = reinterpret_cast<const float*>(smem + ly.dt);
+  const T* s_uc = reinterpret_cast<const T*>(smem + ly.uc);
+  const float4* s_bc = reinterpret_cast<const float4*>(smem + ly.bc);
+  T* s_out = reinterpret_cast<T*>(smem + ly.out);
   const int nchunks = (p.L + kScanTC - 1) / kScanTC;
+  // this thread's row piece: row td, columns 4 pd .. 4 pd + 3 of the CTA's channels
+  ScanPiece pc;
+  const int quads = CH >> 2;
+  pc.live = threadIdx.x < kScanTC * quads;
+  const int td = pc.live ? threadIdx.x / quads : 0;
+  const int pd = pc.live ? threadIdx.x % quads : 0;
+  pc.soff = td * pitch + 4 * pd;
+  pc.goff = (static_cast<long long>(b) * p.L + td) * p.Di + c0 + 4 * pd;
+  pc.uoff = (static_cast<long long>(b) * p.L + td) * uc_parts<T>() * p.Di + c0 + 4 * pd;
 
-  scan_load_chunk<T, SPT>(p, s, 0, b, c0, 0, min(kScanTC, p.L));
+  scan_load_chunk<T>(p, smem, ly, pc, td, 0, b, 0);
+  cp_async_commit();
+  if (nchunks > 1) scan_load_chunk<T>(p, smem, ly, pc, td, 1, b, kScanTC);
   cp_async_commit();
 
   for (int ck = 0; ck < nchunks; ++ck) {
-    const int buf = ck & 1;
-    const int t0 = ck * kScanTC;
-    const int nt = min(kScanTC, p.L - t0);
-    if (ck + 1 < nchunks) {
-      const int t1 = t0 + kScanTC;
-      scan_load_chunk<T, SPT>(p, s, buf ^ 1, b, c0, t1, min(kScanTC, p.L - t1));
-    }
+    const int st = ck % kScanStages, ob = ck & 1;
+    cp_async_wait<1>();          // chunk ck has landed (this thread's copies)
+    __syncthreads();             // ... everyone's; chunk ck-1 fully consumed
+    if (ck > 0) scan_write_piece<T>(p, s_out + (ob ^ 1) * kScanTC * pitch, pc, td, (ck - 1) * kScanTC, kScanTC);
+    if (ck + 2 < nchunks) scan_load_chunk<T>(p, smem, ly, pc, td, (ck + 2) % kScanStages, b, (ck + 2) * kScanTC);
     cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    // prepass: (dt, dt * uc) and D * uc per (token, channel); the thread's
-    // channel is the same on every iteration (kScanThreads % CH == 0)
-    {
-      const int cc = threadIdx.x % CH;
-      const float Dcc = p.D[c0 + cc];
-      for (int t = threadIdx.x / CH; t < kScanTC; t += kScanThreads / CH) {
-        const float d = s.dt[buf][t][cc];
-        const float uu = uc_value<T, SPT>(s, buf, t, cc);
-        s.dtdu[t][cc] = make_float2(d, d * uu);
-        s.dx[t][cc] = Dcc * uu;
-      }
-    }
-    __syncthreads();
 
+    const float* dtc = s_dt + st * kScanTC * pitch + col;
+    const T* ucc = s_uc + st * uc_parts<T>() * kScanTC * pitch + col;
+    const float4* bcc = s_bc + st * (kScanTC / 2) * 16 + q;
+#pragma unroll 2
+    for (int g = 0; g < kScanTC; g += 8) {
+      // this lane's token g+q: dt, uc, dt*uc
+      const int tq = g + q;
+      const float dq = dtc[tq * pitch];
+      float uq;
+      if constexpr (sizeof(T) == 2) uq = to_f32(ucc[tq * pitch]) + to_f32(ucc[(kScanTC + tq) * pitch]);
+      else uq = ucc[tq * pitch];
+      const float duq = dq * uq;
+      float v[8];
 #pragma unroll
-    for (int tg = 0; tg < kScanTC; tg += kScanPG) {
-      // phase 1: decays and inputs of the group's tokens
-      float da[kScanPG][SPT], bu[kScanPG][SPT], cv[kScanPG][SPT];
-#pragma unroll
-      for (int i = 0; i < kScanPG; ++i) {
-        const int t = tg + i;
-        const float2 dd = s.dtdu[t][cl];
-        float bc[2 * SPT];
-#pragma unroll
-        for (int j = 0; j < 2 * SPT; j += 4)
-          *reinterpret_cast<float4*>(&bc[j]) = *reinterpret_cast<const float4*>(&s.bcq[buf][t][q][j]);
-#pragma unroll
-        for (int j = 0; j < SPT; ++j) {
-          da[i][j] = ex2_approx(dd.x * a2[j]);
-          bu[i][j] = dd.y * bc[j];
-          cv[i][j] = bc[SPT + j];
-        }
+      for (int i = 0; i < 8; i += 2) {
+        const int pr = (g + i) >> 1;                          // token pair (g+i, g+i+1)
+        const int src = 4 * i + (lane & 3);                  // lane holding token g+i of this channel
+        const float2 dtp = make_float2(__shfl_sync(0xffffffffu, dq, src), __shfl_sync(0xffffffffu, dq, src + 4));
+        const float2 dup = make_float2(__shfl_sync(0xffffffffu, duq, src), __shfl_sync(0xffffffffu, duq, src + 4));
+        const float4 bb = bcc[pr * 16];                        // B(t,2q) B(t+1,2q) B(t,2q+1) B(t+1,2q+1)
+        const float4 cc = bcc[pr * 16 + 8];                    // the same for C
+        const float2 x0 = mul2(dtp, make_float2(a2_0, a2_0));
+        const float2 x1 = mul2(dtp, make_float2(a2_1, a2_1));
+        const float2 bu0 = mul2(dup, make_float2(bb.x, bb.y));
+        const float2 bu1 = mul2(dup, make_float2(bb.z, bb.w));
+        const float h0a = fmaf(ex2_approx(x0.x), h0, bu0.x);
+        h0 = fmaf(ex2_approx(x0.y), h0a, bu0.y);
+        const float h1a = fmaf(ex2_approx(x1.x), h1, bu1.x);
+        h1 = fmaf(ex2_approx(x1.y), h1a, bu1.y);
+        const float2 pr2 = fma2(make_float2(cc.z, cc.w), make_float2(h1a, h1),
+                                mul2(make_float2(cc.x, cc.y), make_float2(h0a, h0)));
+        v[i] = pr2.x;
+        v[i + 1] = pr2.y;
       }
-      // phase 2: the recurrence and this lane's share of each readout
-      float part[kScanPG];
-#pragma unroll
-      for (int i = 0; i < kScanPG; ++i) {
-        float acc = 0.0f;
-#pragma unroll
-        for (int j = 0; j < SPT; ++j) {
-          h[j] = fmaf(da[i][j], h[j], bu[i][j]);
-          acc = fmaf(cv[i][j], h[j], acc);
-        }
-        part[i] = acc;
-      }
-      // readout: reduce-scatter over the channel's lanes, LANES tokens at a time
-#pragma unroll
-      for (int r0 = 0; r0 < kScanPG; r0 += LANES) {
-        float v[LANES];
-#pragma unroll
-        for (int i = 0; i < LANES; ++i) v[i] = part[r0 + i];
-        const float y = reduce_scatter<LANES>(v, q);
-        const int t = tg + r0 + q;
-        s.out[t][cl] = from_f32<T>(y + s.dx[t][cl]);
-      }
+      const float y = fmaf(Dc, uq, reduce_scatter8(v, q));
+      if (active) s_out[(ob * kScanTC + tq) * pitch + col] = from_f32<T>(y);
     }
-    __syncthreads();
-    // coalesced write-out of the chunk's readout rows
-    {
-      constexpr int PIECES = CH * sizeof(T) / 16;
-      const long long row0 = static_cast<long long>(b) * p.L + t0;
-      for (int i = threadIdx.x; i < nt * PIECES; i += kScanThreads) {
-        const int t = i / PIECES, piece = i % PIECES;
-        *reinterpret_cast<uint4*>(p.M + (row0 + t) * p.Di + c0 + piece * (16 / sizeof(T))) =
-            *reinterpret_cast<const uint4*>(&s.out[t][piece * (16 / sizeof(T))]);
-      }
-    }
-    // the next chunk's prefetch overwrites buf only after its first barrier,
-    // which every thread reaches after finishing this write-out
+  }
+  __syncthreads();
+  {
+    const int ck = nchunks - 1;
+    scan_write_piece<T>(p, s_out + (ck & 1) * kScanTC * pitch, pc, td, ck * kScanTC, p.L - ck * kScanTC);
   }
 
-#pragma unroll
-  for (int j = 0; j < SPT; ++j) p.h[(static_cast<long long>(b) * p.Di + c) * kN + q * SPT + j] = h[j];
+  if (active) {
+    hp[0] = h0;
+    hp[1] = h1;
+  }
   // new conv state: the last K raw inputs (older ones from the previous state
   // when the prompt is shorter than K)
-  if (q == 0) {
+  if (active && q == 0) {
     T* cs = p.conv_state + (static_cast<long long>(b) * p.Di + c) * kK;
     T nw[kK];
 #pragma unroll

@@ -216,6 +216,10 @@ struct GemmArgs {
   int tma_epi;        // row-major gate / residual / softplus epilogue through TMA
                       // (aux tile in, output tile out); set by the host when the
                       // output's columns come in whole 64 (bf16) / 32 (f32) blocks
+  int full_tiles;     // tail_nsplit > 1: work units [0, full_tiles) are whole tiles,
+  int tail_nsplit;    // and every later tile is cut along N into tail_nsplit units
+                      // of BN / tail_nsplit columns (wave quantisation: the last,
+                      // partial wave of tiles spreads over more SMs; no K split)
 };
 
 // The final op on one element.  `o` is the output's linear index, `a` the aux
@@ -385,24 +389,40 @@ struct Cfg {
 
 struct TileCoord {
   int m, n, split, kb0, kb1;
+  int n0, bn;          // first output column and width of this unit
 };
 
+template <int BN>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   TileCoord c;
+  if (g.tail_nsplit > 1 && t >= g.full_tiles) {
+    const int r = t - g.full_tiles;
+    const int tile = g.full_tiles + r / g.tail_nsplit;
+    c.m = tile % g.m_tiles;
+    c.n = tile / g.m_tiles;
+    c.bn = BN / g.tail_nsplit;
+    c.n0 = c.n * BN + (r % g.tail_nsplit) * c.bn;
+    c.split = 0;
+    c.kb0 = 0;
+    c.kb1 = g.k_blocks;
+    return c;
+  }
   c.m = t % g.m_tiles;
   const int r = t / g.m_tiles;
   c.n = r % g.n_tiles;
   c.split = r / g.n_tiles;
   c.kb0 = c.split * g.kb_per_split;
   c.kb1 = min(g.k_blocks, c.kb0 + g.kb_per_split);
+  c.n0 = c.n * BN;
+  c.bn = BN;
   return c;
 }
 
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmAux, const __grid_constant__ CUtensorMap tmOut,
-                   const GemmArgs g) {
+                   const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmAux,
+                   const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -443,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (g.tail_nsplit > 1 && !B_MN) prefetch_tmap(&tmB2);
     if (C::kTmaEpi && g.tma_epi) {
       if (KIND != EPI_SOFTPLUS && g.aux != nullptr) prefetch_tmap(&tmAux);
       prefetch_tmap(&tmOut);
@@ -468,10 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;  // per stage: outstanding load, its parity
       bool ok = true;
       for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord(g, t);
+        const TileCoord c = tile_coord<BN>(g, t);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], C::kABytes + c.bn * BK * 2);
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
           if (A_MN) {  // [K, M] in memory: boxes of 64 m x 64 k
@@ -484,9 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (B_MN) {  // [K, N]: BN/64 boxes of 64 n x 64 k
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(b_dst + j * 8192, &tmB, &full[stage], c.n * BN + 64 * j, kb_b);
-          } else {     // [N, K]: one box of 64 k x BN n
-            tma_load_2d(b_dst, &tmB, &full[stage], kb_b, c.n * BN);
+              if (64 * j < c.bn) tma_load_2d(b_dst + j * 8192, &tmB, &full[stage], c.n0 + 64 * j, kb_b);
+          } else {     // [N, K]: one box of 64 k x BN n (tail units: 64 k x bn n)
+            tma_load_2d(b_dst, c.bn == BN ? &tmB : &tmB2, &full[stage], kb_b, c.n0);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -511,10 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord(g, t);
+        const TileCoord c = tile_coord<BN>(g, t);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t idesc = c.bn == BN ? C::kIdesc : idesc_bf16(BM, c.bn, A_MN, B_MN);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -526,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                      : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, C::kIdesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -550,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t aux_phase = 0;    // parity bit per aux slot
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     for (int t = blockIdx.x; t < g.tiles; t += gridDim.x) {
-      const TileCoord c = tile_coord(g, t);
+      const TileCoord c = tile_coord<BN>(g, t);
       const bool split = g.splits > 1 && KIND != EPI_F32_PARTIAL;
       const bool tma = C::kTmaEpi && g.tma_epi && !split;
       if (tma) {
@@ -560,16 +582,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (has_aux && ep_tid == 0) {
 #pragma unroll
           for (int j = 0; j < C::kSlots; ++j) {
-            const int n0 = c.n * BN + 64 * j;
-            if (n0 < g.N) {
+            const int n0 = c.n0 + 64 * j;
+            if (64 * j < c.bn && n0 < g.N) {
               mbar_arrive_expect_tx(&auxf[j], kSlotBytes);
               tma_load_2d(epi_area + j * kSlotBytes, &tmAux, &auxf[j], n0, c.m * BM);
             }
           }
         }
         if (KIND == EPI_SOFTPLUS)
-          for (int i = ep_tid; i < BN; i += 128)
-            epi_vec[i] = c.n * BN + i < g.N ? g.vec[c.n * BN + i] : 0.0f;
+          for (int i = ep_tid; i < c.bn; i += 128)
+            epi_vec[i] = c.n0 + i < g.N ? g.vec[c.n0 + i] : 0.0f;
       }
       bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
       // the split-K and TMA paths synchronise the 4 epilogue warps, so they must
@@ -586,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = quarter * 32 + lane;
         if (KIND == EPI_SOFTPLUS) {
 #pragma unroll 1
-          for (int ch = 0; ch < BN / 32; ++ch) {
-            const int n0 = c.n * BN + 32 * ch;
+          for (int ch = 0; ch < c.bn / 32; ++ch) {
+            const int n0 = c.n0 + 32 * ch;
             if (n0 >= g.N) break;
             uint8_t* blk = epi_area + (ch & 1) * kSlotBytes;
             if (ch >= 2) {            // this slot's store from two chunks ago has read it
@@ -616,8 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll 1
           for (int j = 0; j < C::kSlots; ++j) {
-            const int n0 = c.n * BN + 64 * j;
-            if (n0 >= g.N) break;
+            const int n0 = c.n0 + 64 * j;
+            if (64 * j >= c.bn || n0 >= g.N) break;
             uint8_t* blk = epi_area + j * kSlotBytes;
             if (has_aux) {
               ok = mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag);
@@ -675,13 +697,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = 0; ch < c.bn / 32; ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + ch * 32, r);
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        const int n0 = c.n * BN + ch * 32;
+        const int n0 = c.n0 + ch * 32;
         if (split) {
           // this split's partial tile, summed in split order by the last CTA
           float* part = g.partials + static_cast<long long>(c.split) * g.split_stride;
@@ -726,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
 #pragma unroll 1
           for (int ch = 0; ch < BN / 32; ++ch) {
-            const int n0 = c.n * BN + ch * 32;
+            const int n0 = c.n0 + ch * 32;
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;

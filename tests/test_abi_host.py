@@ -58,16 +58,18 @@ def test_workspace_queries(lib):
     # (9 splits for 16 row tiles over 160 k-blocks; 54 splits of 3 k-blocks for
     # one row tile)
     # + xdbl + split delta (bf16, 2 x dt_rank padded to 192) + dt (f32)
+    # + B | C regrouped into token pairs (64 floats per pair)
     Rp = 192
     want = (r256(T * Di * 4) + r256(9 * T * ldx * 4) + r256(T * ldx * 4) + r256(T * 2 * Rp * 2)
-            + r256(T * Di * 4))
+            + r256(T * Di * 4) + r256(T // 2 * 64 * 4))
     assert abi.sambay_scan_prefill_workspace(d) == want
     assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == \
         r256(64 * Di * 4) + r256(54 * 64 * ldx * 4) + r256(64 * ldx * 4) + r256(64 * 2 * Rp * 2) \
-        + r256(64 * Di * 4)
+        + r256(64 * Di * 4) + r256(64 * 64 * 4)
     # float32 mode: no partials, no split delta
     f = abi.make_dims(1, 64, 64, 128, 16, 4, 4, abi.F32)
-    assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4)
+    assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4) \
+        + r256(32 * 64 * 4)
     assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2)
     assert abi.gmu_step_workspace(d, 64) > 64 * 5120 * 2
     # invalid or unsupported dims -> 0
