@@ -34,10 +34,9 @@ sys.path.insert(0, ROOT)
 from gated_memory_sharing_b200 import synth  # noqa: E402
 
 WORKLOAD = "prefill_b1_l2048"
-# DRAM bytes (read + write) per launch of a kernel, from one ncu capture of the
-# benchmarked workload (profiles/); None once the kernel has changed since.
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the current kernels,
-# from profiles/ (empty until captured again after a kernel change)
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# kernel, from one ncu capture of the benchmarked workload (profiles/); a kernel
+# changed since its capture has no entry (reported as null).
 DRAM_TRAFFIC = {}
 METRIC = "scan+GMU prefill tokens/s"
 UNIT = "tokens/s"
