@@ -51,17 +51,14 @@ __device__ __forceinline__ float lg2_approx(float x) {
 // log1p(y): for y < 1/16 its Taylor series y - y^2/2 + y^3/3 - y^4/4 + y^5/5
 // (the first omitted term is below 2e-7 of the sum); otherwise
 // log2(1 + y) * ln 2 with 1 + y >= 1.0625, where the SFU's absolute error in
-// log2 is a few 1e-7 of the result.  No cut-over to x is needed: for large x,
-// y underflows towards 0 and the series returns y.
+// log2 is a few 1e-7 of the result.  Both are evaluated and one selected, so
+// a warp whose lanes straddle 1/16 does not run the two paths one after the
+// other.  For large x, y underflows towards 0 and the series returns y.
 __device__ __forceinline__ float softplus(float x) {
   const float y = ex2_approx(-fabsf(x) * kLog2e);
-  float l;
-  if (y < 0.0625f) {
-    l = y * fmaf(-y, fmaf(-y, fmaf(-y, fmaf(-y, 0.2f, 0.25f), 0.33333334f), 0.5f), 1.0f);
-  } else {
-    l = lg2_approx(1.0f + y) * kLn2;
-  }
-  return fmaxf(x, 0.0f) + l;
+  const float series = y * fmaf(-y, fmaf(-y, fmaf(-y, fmaf(-y, 0.2f, 0.25f), 0.33333334f), 0.5f), 1.0f);
+  const float viaLog = lg2_approx(1.0f + y) * kLn2;
+  return fmaxf(x, 0.0f) + (y < 0.0625f ? series : viaLog);
 }
 
 // Pack / unpack helpers for 16-byte vector access.

@@ -287,13 +287,13 @@ TailPlan tail_plan(int tiles, int BN, int sms) {
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
 // split_count for the same sizes); `balance_tail` (no K split) applies
 // tail_plan.
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
                      sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false) {
   using namespace sambay::tc;
-  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW>;
   static bool attr_set[kMaxDevices] = {};
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS>;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS, EW>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem)) != cudaSuccess)
@@ -345,7 +345,7 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   const int grid = std::min(g.tiles, sms);
   {
     ProfScope ps(name, st);
-    kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
+    kern<<<grid, gemm_threads(EW), C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -443,7 +443,7 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     if (rows <= sambay::tc::BM)   // one row tile (decode): narrower tiles, more CTAs
       SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
     else
-      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
+      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
     SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
@@ -706,10 +706,10 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   const int Dm = d->d_model, Di = d->d_inner, T = static_cast<int>(rows);
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
-  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false>(
+  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
-  SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false>(
+  SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false, 8>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st, true)));
   return SAMBAY_OK;

@@ -3,7 +3,9 @@
 // epilogues.  One CTA per SM; warp roles:
 //   warp 0        TMA producer (one lane): A and B tiles into a smem ring
 //   warp 1        MMA issuer (one lane) + TMEM owner (whole warp allocates)
-//   warps 2..5    epilogue: tcgen05.ld TMEM -> registers -> fused op -> HBM
+//   warps 2..     EW epilogue warps (4 or 8): tcgen05.ld TMEM -> registers ->
+//                 fused op -> HBM.  Warp w reads TMEM lanes 32 (w % 4) ..; with
+//                 8, the two warps of a lane quarter take alternate column blocks
 // The accumulator is double-buffered in TMEM so the epilogue of one tile
 // overlaps the main loop of the next.  No cluster multicast is used: every
 // CTA loads its own tiles.
@@ -28,7 +30,7 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                       // one 128-byte swizzle atom of bf16
-constexpr int kThreads = 192;                // 6 warps
+__host__ __device__ constexpr int gemm_threads(int EW) { return 64 + 32 * EW; }
 constexpr unsigned long long kWaitCycles = 1ull << 34;  // ~8 s at 2 GHz
 constexpr unsigned long long kDrainCycles = 1ull << 28;
 
@@ -152,18 +154,25 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// AND of a predicate over the 128 epilogue threads (named barrier 1).
+// AND of a predicate over the NT epilogue threads (named barrier 1).
+template <int NT>
 __device__ __forceinline__ bool epi_agree(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(r)
-      : "r"(ok ? 1u : 0u)
+      : "r"(ok ? 1u : 0u), "n"(NT)
       : "memory");
   return r != 0;
+}
+
+// barrier over the NT epilogue threads (named barrier 1)
+template <int NT>
+__device__ __forceinline__ void named_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
 // Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 format (version 1).
@@ -362,17 +371,19 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row0, int lane,
 constexpr int kSlotBytes = 16384;             // one 128-row x 128-byte epilogue block
 constexpr int kMaxDynSmem = 232448;           // 227 KB per CTA on sm_100
 
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW>
 struct Cfg {
   static constexpr int kABytes = BM * BK * 2;   // 16 KB
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   // TMA epilogue: bf16 outputs keep one 128 x 64 block per 64 output columns
   // (the whole tile's aux arrives ahead of the accumulator); f32 outputs
-  // double-buffer 128 x 32 blocks
+  // double-buffer 128 x 32 blocks per group of 4 epilogue warps
+  static constexpr int kHalves = EW / 4;
   static constexpr bool kTmaEpi = !TRANS && (KIND == EPI_GATE || KIND == EPI_RESID || KIND == EPI_SOFTPLUS);
-  static constexpr int kSlots = !kTmaEpi ? 0 : (KIND == EPI_SOFTPLUS ? 2 : BN / 64);
-  static constexpr int kEpiBytes = kTmaEpi ? kSlots * kSlotBytes + 1024 /*bias*/ : 4 * kEpiWarpBytes;
+  static constexpr int kSlots = !kTmaEpi ? 0 : (KIND == EPI_SOFTPLUS ? 2 * kHalves : BN / 64);
+  static constexpr int kStageArea = kSlots * kSlotBytes > EW * kEpiWarpBytes ? kSlots * kSlotBytes : EW * kEpiWarpBytes;
+  static constexpr int kEpiBytes = kStageArea + (kTmaEpi ? 1024 /*bias*/ : 0);
   static constexpr int kFixed = 1024 /*align slack*/ + 512 /*barriers*/ + kEpiBytes;
   static constexpr int kStagesFit = (kMaxDynSmem - kFixed) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -382,7 +393,7 @@ struct Cfg {
   static constexpr size_t kSmem = static_cast<size_t>(kFixed) + static_cast<size_t>(kStages) * kStageBytes;
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
-  static_assert(kSlots * kSlotBytes >= (kTmaEpi ? 4 * kEpiWarpBytes : 0), "fallback staging fits the slots");
+  static_assert(EW == 4 || EW == 8, "one or two epilogue warps per TMEM lane quarter");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, whole 32-column epilogue chunks");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element atoms");
 };
@@ -418,12 +429,12 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   return c;
 }
 
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW>
+__global__ void __launch_bounds__(gemm_threads(EW), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmAux,
                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
-  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
@@ -440,8 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxf + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;
-  uint8_t* epi_stage = epi_area;                           // fallback staging, 4 x kEpiWarpBytes
-  float* epi_vec = reinterpret_cast<float*>(epi_area + C::kSlots * kSlotBytes);  // tile's bias
+  uint8_t* epi_stage = epi_area;                           // fallback staging, EW x kEpiWarpBytes
+  float* epi_vec = reinterpret_cast<float*>(epi_area + C::kStageArea);  // tile's bias
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -453,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], EW);
     }
     mbar_init(drain, 1);
     for (int j = 0; j < 4; ++j) mbar_init(&auxf[j], 1);
@@ -564,12 +575,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ epilogue
+    constexpr int H = C::kHalves;            // epilogue warps per TMEM lane quarter
+    constexpr int EPI_THREADS = 32 * EW;
     const int quarter = warp & 3;            // TMEM lanes [32*quarter, +32)
-    const int ep_tid = threadIdx.x - 64;     // 0..127
+    const int ep_tid = threadIdx.x - 64;     // 0 .. 32*EW - 1
+    const int half = (warp - 2) / 4;         // which of the quarter's warps: column blocks half, half + H, ...
     uint8_t* my_stage = epi_stage + (warp - 2) * kEpiWarpBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t aux_phase = 0;    // parity bit per aux slot
+    int sp_local = 0;          // softplus chunks this warp has staged (slot double buffering)
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     for (int t = blockIdx.x; t < g.tiles; t += gridDim.x) {
       const TileCoord c = tile_coord<BN>(g, t);
@@ -590,13 +605,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (KIND == EPI_SOFTPLUS)
-          for (int i = ep_tid; i < c.bn; i += 128)
+          for (int i = ep_tid; i < c.bn; i += EPI_THREADS)
             epi_vec[i] = c.n0 + i < g.N ? g.vec[c.n0 + i] : 0.0f;
       }
       bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
-      // the split-K and TMA paths synchronise the 4 epilogue warps, so they must
+      // the split-K and TMA paths synchronise the epilogue warps, so they must
       // agree on leaving the loop together (the barrier also publishes epi_vec)
-      if (split || tma) ok = epi_agree(ok);
+      if (split || tma) ok = epi_agree<EPI_THREADS>(ok);
       if (!ok) break;
       tc_fence_after();
       const int row = c.m * BM + quarter * 32 + lane;
@@ -608,14 +623,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = quarter * 32 + lane;
         if (KIND == EPI_SOFTPLUS) {
 #pragma unroll 1
-          for (int ch = 0; ch < c.bn / 32; ++ch) {
+          for (int ch = half; ch < c.bn / 32; ch += H) {
             const int n0 = c.n0 + 32 * ch;
             if (n0 >= g.N) break;
-            uint8_t* blk = epi_area + (ch & 1) * kSlotBytes;
-            if (ch >= 2) {            // this slot's store from two chunks ago has read it
+            uint8_t* blk = epi_area + (half * 2 + (sp_local & 1)) * kSlotBytes;
+            if (sp_local >= 2) {      // this slot's store from two chunks ago has read it
               if (lane == 0) bulk_wait_read<1>();
               __syncwarp();
             }
+            ++sp_local;
             uint32_t rr[32];
             tmem_ld_32x32b_x32(t_row + 32 * ch, rr);
 #pragma unroll
@@ -636,17 +652,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          // slot j (64 columns) goes to the quarter's warp j % H; every warp runs
+          // the same number of rounds, since each round ends in a barrier
 #pragma unroll 1
-          for (int j = 0; j < C::kSlots; ++j) {
+          for (int j0 = 0; j0 < C::kSlots; j0 += H) {
+            const int j = j0 + half;
             const int n0 = c.n0 + 64 * j;
-            if (64 * j >= c.bn || n0 >= g.N) break;
-            uint8_t* blk = epi_area + j * kSlotBytes;
+            const bool mine = j < C::kSlots && 64 * j < c.bn && n0 < g.N;
             if (has_aux) {
-              ok = mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag);
-              ok = epi_agree(ok);
+              ok = mine ? mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag) : true;
+              ok = epi_agree<EPI_THREADS>(ok);
               if (!ok) break;
-              aux_phase ^= 1u << j;
+              if (mine) aux_phase ^= 1u << j;
             }
+            if (!mine) continue;
+            uint8_t* blk = epi_area + j * kSlotBytes;
 #pragma unroll 1
             for (int h = 0; h < 2; ++h) {
               uint32_t rr[32];
@@ -693,11 +713,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // aux loads and bias overwrite them
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        sp_local = 0;
+        named_bar_sync<EPI_THREADS>();
         continue;
       }
 #pragma unroll 1
-      for (int ch = 0; ch < c.bn / 32; ++ch) {
+      for (int ch = half; ch < c.bn / 32; ch += H) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + ch * 32, r);
         float v[32];
@@ -735,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The last CTA to finish a split-K tile sums the partials in split
         // order (deterministic), applies the final op and resets the counter.
         __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        named_bar_sync<EPI_THREADS>();
         if (ep_tid == 0) {
           const int tile_mn = c.m + g.m_tiles * c.n;
           const int prev = atomicAdd(g.counters + tile_mn, 1);
@@ -743,11 +764,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last) g.counters[tile_mn] = 0;
           *last_flag = last;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        named_bar_sync<EPI_THREADS>();
         if (*last_flag) {
           __threadfence();
 #pragma unroll 1
-          for (int ch = 0; ch < BN / 32; ++ch) {
+          for (int ch = half; ch < BN / 32; ch += H) {
             const int n0 = c.n0 + ch * 32;
             float v[32];
 #pragma unroll
@@ -770,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             epi_chunk<KIND, TRANS>(g, row - lane, lane, n0, v, my_stage);
           }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        named_bar_sync<EPI_THREADS>();
       }
     }
   }
