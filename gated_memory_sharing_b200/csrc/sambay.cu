@@ -709,7 +709,7 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
-  SAMBAY_TRY((run_tc<128, false, true, sambay::tc::EPI_RESID, false, 8>(
+  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st, true)));
   return SAMBAY_OK;
