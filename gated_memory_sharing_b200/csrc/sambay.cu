@@ -271,13 +271,13 @@ struct TailPlan {
   int full, nsplit;
 };
 
-TailPlan tail_plan(int tiles, int BN, int sms) {
+TailPlan tail_plan(int tiles, int BN, int slots, int min_width) {
   TailPlan tp{tiles, 1};
-  const int waves = tiles / sms, tail = tiles % sms;
+  const int waves = tiles / slots, tail = tiles % slots;
   if (waves == 0 || tail == 0) return tp;
-  for (int cand = BN / 64; cand >= 2; cand /= 2)
-    if (BN % (cand * 64) == 0 && tail * cand <= sms) {
-      tp.full = waves * sms;
+  for (int cand = BN / min_width; cand >= 2; cand /= 2)
+    if (BN % (cand * min_width) == 0 && tail * cand <= slots) {
+      tp.full = waves * slots;
       tp.nsplit = cand;
       break;
     }
@@ -286,24 +286,42 @@ TailPlan tail_plan(int tiles, int BN, int sms) {
 
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
 // split_count for the same sizes); `balance_tail` (no K split) applies
-// tail_plan.
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4>
+// tail_plan.  PAIR: 256-row tiles on CTA pairs (clusters of two).
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4, bool PAIR = false>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
                      sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false) {
   using namespace sambay::tc;
-  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   static bool attr_set[kMaxDevices] = {};
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS, EW>;
+  static int pair_slots[kMaxDevices] = {};   // co-resident clusters of two (PAIR)
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem)) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
+    if (PAIR) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * (sms / 2));
+      q.blockDim = dim3(gemm_threads(EW));
+      q.dynamicSmemBytes = C::kSmem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n < 1) return SAMBAY_ERR_CUDA;
+      pair_slots[dev] = n;
+    }
     attr_set[dev] = true;
   }
   CUtensorMap ta, tb;
   // A K-major: [M, K] -> box {64 k, 128 m};  MN-major: [K, M] -> box {64 m, 64 k}
+  // B K-major: [N, K] -> box {64 k, kBHalf n} (a pair's CTA loads half the tile's columns)
   if (!make_map(&ta, a.ptr, a.cols, a.rows, a.cols * 2, A_MN ? 64 : BM)) return SAMBAY_ERR_CUDA;
-  if (!make_map(&tb, b.ptr, b.cols, b.rows, b.cols * 2, B_MN ? 64 : BN)) return SAMBAY_ERR_CUDA;
+  if (!make_map(&tb, b.ptr, b.cols, b.rows, b.cols * 2, B_MN ? 64 : C::kBHalf)) return SAMBAY_ERR_CUDA;
   // row-major epilogue through TMA when the output columns come in whole
   // blocks: bf16 outputs in 64-column blocks (aux in 128 x 64 boxes, stores in
   // 32 x 64 boxes per warp), f32 outputs in 32 x 32 boxes
@@ -323,7 +341,7 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
       g.tma_epi = 1;
     }
   }
-  g.m_tiles = (g.M + BM - 1) / BM;
+  g.m_tiles = (g.M + C::kBMT - 1) / C::kBMT;
   g.n_tiles = (g.N + BN - 1) / BN;
   g.k_blocks = (g.K + BK - 1) / BK;
   splits = std::max(1, std::min(splits, g.k_blocks));
@@ -333,19 +351,39 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   g.full_tiles = g.tiles;
   g.tail_nsplit = 1;
   CUtensorMap tb2 = tb;
+  const int slots = PAIR ? pair_slots[dev] : sms;   // work units in flight at once
   if (balance_tail && g.splits == 1) {
-    const TailPlan tp = tail_plan(g.tiles, BN, sms);
+    // narrowest unit: 64 columns per CTA's B load (MN-major B: whole 64-column boxes)
+    const int min_width = (PAIR && B_MN) ? 128 : 64;
+    const TailPlan tp = tail_plan(g.tiles, BN, slots, min_width);
     if (tp.nsplit > 1) {
-      if (!B_MN && !make_map(&tb2, b.ptr, b.cols, b.rows, b.cols * 2, BN / tp.nsplit)) return SAMBAY_ERR_CUDA;
+      const int hb = (BN / tp.nsplit) / (PAIR ? 2 : 1);
+      if (!B_MN && !make_map(&tb2, b.ptr, b.cols, b.rows, b.cols * 2, hb)) return SAMBAY_ERR_CUDA;
       g.tiles = tp.full + (g.tiles - tp.full) * tp.nsplit;
       g.full_tiles = tp.full;
       g.tail_nsplit = tp.nsplit;
     }
   }
-  const int grid = std::min(g.tiles, sms);
+  const int units = std::min(g.tiles, slots);
   {
     ProfScope ps(name, st);
-    kern<<<grid, gemm_threads(EW), C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
+    if (PAIR) {
+      cudaLaunchConfig_t lc = {};
+      lc.gridDim = dim3(2 * units);
+      lc.blockDim = dim3(gemm_threads(EW));
+      lc.dynamicSmemBytes = C::kSmem;
+      lc.stream = st;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      lc.attrs = at;
+      lc.numAttrs = 1;
+      if (cudaLaunchKernelEx(&lc, kern, ta, tb, tb2, taux, tout, g) != cudaSuccess) return SAMBAY_ERR_CUDA;
+    } else {
+      kern<<<units, gemm_threads(EW), C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
+    }
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -706,10 +744,10 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   const int Dm = d->d_model, Di = d->d_inner, T = static_cast<int>(rows);
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
-  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8>(
+  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8, true>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
-  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8>(
+  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8, true>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st, true)));
   return SAMBAY_OK;

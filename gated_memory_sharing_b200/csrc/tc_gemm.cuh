@@ -7,8 +7,17 @@
 //                 fused op -> HBM.  Warp w reads TMEM lanes 32 (w % 4) ..; with
 //                 8, the two warps of a lane quarter take alternate column blocks
 // The accumulator is double-buffered in TMEM so the epilogue of one tile
-// overlaps the main loop of the next.  No cluster multicast is used: every
-// CTA loads its own tiles.
+// overlaps the main loop of the next.  No TMA multicast is used: every CTA
+// loads its own tiles.
+//
+// PAIR mode (cta_group::2): a cluster of two CTAs on two SMs computes one
+// 256 x BN tile.  Each CTA loads its own 128 rows of A and its half of B (BN/2
+// columns), so a pair moves half the B bytes per flop of two 128 x BN tiles;
+// the leader CTA (rank 0) issues the M = 256 MMAs, which read both CTAs'
+// shared memory and write each CTA's 128 accumulator rows into that CTA's
+// TMEM.  Both CTAs' TMA loads complete on the leader's stage barriers, the
+// leader's commits arrive on both CTAs' barriers, and both CTAs' epilogue
+// warps hand the accumulator back through the leader's barrier.
 //
 // D[m, n] = sum_k A[m, k] * B[k, n]
 //   A: K-major ([M, K], k contiguous) or MN-major ([K, M], m contiguous)
@@ -92,6 +101,33 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// ---- CTA-pair (cta_group::2) forms.  A shared::cta address with the peer
+// bit cleared names the same variable in the pair's rank-0 CTA.
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose bytes complete on the
+// leader CTA's barrier
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & kPeerBitMask), "r"(c0), "r"(c1)
+      : "memory");
+}
+// arrive on the leader CTA's copy of this barrier
+__device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(smem_u32(bar) & kPeerBitMask) : "memory");
+}
+
 // shared -> global tile store (bulk group); out-of-range rows/columns are clipped
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
   asm volatile(
@@ -125,6 +161,32 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
+      : "memory");
+}
+
+// the MMAs issued so far by this thread, once complete, arrive on the barrier
+// at this offset in both CTAs of the pair
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// the same, for MMAs issued with cta_group::2, arriving on this CTA only
+__device__ __forceinline__ void tc_commit2(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -371,10 +433,12 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row0, int lane,
 constexpr int kSlotBytes = 16384;             // one 128-row x 128-byte epilogue block
 constexpr int kMaxDynSmem = 232448;           // 227 KB per CTA on sm_100
 
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW>
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW, bool PAIR>
 struct Cfg {
+  static constexpr int kBMT = PAIR ? 2 * BM : BM;   // tile rows (a pair: 128 per CTA)
+  static constexpr int kBHalf = PAIR ? BN / 2 : BN; // B columns this CTA loads per tile
   static constexpr int kABytes = BM * BK * 2;   // 16 KB
-  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kBBytes = kBHalf * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   // TMA epilogue: bf16 outputs keep one 128 x 64 block per 64 output columns
   // (the whole tile's aux arrives ahead of the accumulator); f32 outputs
@@ -389,13 +453,14 @@ struct Cfg {
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
-  static constexpr uint32_t kIdesc = idesc_bf16(BM, BN, A_MN, B_MN);
+  static constexpr uint32_t kIdesc = idesc_bf16(kBMT, BN, A_MN, B_MN);
   static constexpr size_t kSmem = static_cast<size_t>(kFixed) + static_cast<size_t>(kStages) * kStageBytes;
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
   static_assert(EW == 4 || EW == 8, "one or two epilogue warps per TMEM lane quarter");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, whole 32-column epilogue chunks");
-  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-element atoms");
+  static_assert(!B_MN || kBHalf % 64 == 0, "MN-major B tiles are whole 64-element atoms");
+  static_assert(!PAIR || (!TRANS && !A_MN && KIND != EPI_F32_PARTIAL), "pairs serve the row-major prefill GEMMs");
 };
 
 struct TileCoord {
@@ -429,13 +494,17 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   return c;
 }
 
-template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW>
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW, bool PAIR>
 __global__ void __launch_bounds__(gemm_threads(EW), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmAux,
                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
-  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW>;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   constexpr int S = C::kStages;
+  // work units: one per CTA, or one per CTA pair (cluster of 2)
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ustride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -464,7 +533,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], EW);
+      mbar_init(&tempty[a], PAIR ? 2 * EW : EW);
     }
     mbar_init(drain, 1);
     for (int j = 0; j < 4; ++j) mbar_init(&auxf[j], 1);
@@ -481,14 +550,23 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     }
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(C::kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (PAIR) {   // warp 1 of both CTAs: the same columns in each CTA's TMEM
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync();   // the peer's barriers exist before any load or arrive targets them
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -499,34 +577,44 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;  // per stage: outstanding load, its parity
       bool ok = true;
-      for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
+      for (int t = unit0; t < g.tiles && ok; t += ustride) {
         const TileCoord c = tile_coord<BN>(g, t);
+        const int arow = c.m * C::kBMT + rank * BM;       // this CTA's A rows
+        const int hb = PAIR ? c.bn / 2 : c.bn;            // this CTA's B columns
+        const int bcol = c.n0 + rank * hb;
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::kABytes + c.bn * BK * 2);
+          // the leader's barrier counts the bytes of both CTAs of a pair
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], (C::kABytes + hb * BK * 2) * (PAIR ? 2 : 1));
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
+          auto load = [&](void* dst, const CUtensorMap* map, int c0, int c1) {
+            if (PAIR) tma_load_2d_pair(dst, map, &full[stage], c0, c1);
+            else tma_load_2d(dst, map, &full[stage], c0, c1);
+          };
           if (A_MN) {  // [K, M] in memory: boxes of 64 m x 64 k
-            tma_load_2d(a_dst, &tmA, &full[stage], c.m * BM, kb * BK);
-            tma_load_2d(a_dst + 8192, &tmA, &full[stage], c.m * BM + 64, kb * BK);
+            load(a_dst, &tmA, arow, kb * BK);
+            load(a_dst + 8192, &tmA, arow + 64, kb * BK);
           } else {     // [M, K]: one box of 64 k x 128 m
-            tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, c.m * BM);
+            load(a_dst, &tmA, kb * BK, arow);
           }
           const int kb_b = g.b_k_wrap > 0 ? (kb * BK) % g.b_k_wrap : kb * BK;
-          if (B_MN) {  // [K, N]: BN/64 boxes of 64 n x 64 k
+          if (B_MN) {  // [K, N]: boxes of 64 n x 64 k
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              if (64 * j < c.bn) tma_load_2d(b_dst + j * 8192, &tmB, &full[stage], c.n0 + 64 * j, kb_b);
-          } else {     // [N, K]: one box of 64 k x BN n (tail units: 64 k x bn n)
-            tma_load_2d(b_dst, c.bn == BN ? &tmB : &tmB2, &full[stage], kb_b, c.n0);
+            for (int j = 0; j < C::kBHalf / 64; ++j)
+              if (64 * j < hb) load(b_dst + j * 8192, &tmB, bcol + 64 * j, kb_b);
+          } else {     // [N, K]: one box of 64 k x kBHalf n (tail units: 64 k x hb n)
+            load(b_dst, hb == C::kBHalf ? &tmB : &tmB2, kb_b, bcol);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
       }
-      if (*abort_flag) {
+      if (*abort_flag && rank == 0) {
         // drain: every issued load must land before the CTA's smem goes away
+        // (in a pair the leader's barriers count the peer's loads too, and the
+        // peer stays resident until the leader reaches the final cluster barrier)
         for (int s = 0; s < S; ++s)
           if (issued_mask & (1u << s)) {
             volatile int dummy = 0;
@@ -536,18 +624,18 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
+      for (int t = unit0; t < g.tiles && ok; t += ustride) {
         const TileCoord c = tile_coord<BN>(g, t);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        const uint32_t idesc = c.bn == BN ? C::kIdesc : idesc_bf16(BM, c.bn, A_MN, B_MN);
+        const uint32_t idesc = c.bn == BN ? C::kIdesc : idesc_bf16(C::kBMT, c.bn, A_MN, B_MN);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -559,17 +647,21 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
                                      : sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                      : sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+            if (PAIR) tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+            else tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if (PAIR) tc_commit_pair(&empty[stage]);
+          else tc_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if (PAIR) tc_commit_pair(&tfull[acc]);
+        else tc_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // all MMAs issued by this thread complete before TMEM is released
-      tc_commit(drain);
+      if (PAIR) tc_commit2(drain);
+      else tc_commit(drain);
       volatile int dummy = 0;
       mbar_wait(drain, 0, &dummy, kDrainCycles);
     }
@@ -586,8 +678,9 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     uint32_t aux_phase = 0;    // parity bit per aux slot
     int sp_local = 0;          // softplus chunks this warp has staged (slot double buffering)
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
-    for (int t = blockIdx.x; t < g.tiles; t += gridDim.x) {
+    for (int t = unit0; t < g.tiles; t += ustride) {
       const TileCoord c = tile_coord<BN>(g, t);
+      const int arow = c.m * C::kBMT + rank * BM;     // this CTA's first output row
       const bool split = g.splits > 1 && KIND != EPI_F32_PARTIAL;
       const bool tma = C::kTmaEpi && g.tma_epi && !split;
       if (tma) {
@@ -600,7 +693,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
             const int n0 = c.n0 + 64 * j;
             if (64 * j < c.bn && n0 < g.N) {
               mbar_arrive_expect_tx(&auxf[j], kSlotBytes);
-              tma_load_2d(epi_area + j * kSlotBytes, &tmAux, &auxf[j], n0, c.m * BM);
+              tma_load_2d(epi_area + j * kSlotBytes, &tmAux, &auxf[j], n0, arow);
             }
           }
         }
@@ -614,7 +707,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       if (split || tma) ok = epi_agree<EPI_THREADS>(ok);
       if (!ok) break;
       tc_fence_after();
-      const int row = c.m * BM + quarter * 32 + lane;
+      const int row = arow + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       if (tma) {
@@ -647,7 +740,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, c.m * BM + quarter * 32);
+              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, arow + quarter * 32);
               bulk_commit();
             }
           }
@@ -699,7 +792,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, c.m * BM + quarter * 32);
+              tma_store_2d(&tmOut, blk + quarter * 32 * 128, n0, arow + quarter * 32);
               bulk_commit();
             }
           }
@@ -707,7 +800,10 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (lane == 0) {
+          if (PAIR && rank != 0) mbar_arrive_leader(&tempty[acc]);
+          else mbar_arrive(&tempty[acc]);
+        }
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         // every store of this tile has read its slot before the next tile's
         // aux loads and bias overwrite them
@@ -749,7 +845,10 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR && rank != 0) mbar_arrive_leader(&tempty[acc]);
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
       if (split) {
@@ -798,12 +897,20 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
 
   if (C::kTmaEpi && warp >= 2 && lane == 0) bulk_wait_read<0>();   // no store still reading smem
   tc_fence_before();
-  __syncthreads();
+  // a pair ends together: the leader's MMAs write the peer's TMEM and read its
+  // shared memory, and the peer's arrivals target the leader's barriers
+  if (PAIR) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(C::kTmemCols)
-                 : "memory");
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(C::kTmemCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(C::kTmemCols)
+                   : "memory");
   }
 }
 
