@@ -554,12 +554,15 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
                                   static_cast<const T*>(w->conv_w),
                                   static_cast<const T*>(w->conv_b), uc, d->batch, d->seqlen,
                                   d->d_inner, zero_init};
-    constexpr int VEC = 8 / sizeof(T);
-    constexpr int TT = 8;
-    const long long threads =
-        static_cast<long long>(d->batch) * ((d->seqlen + TT - 1) / TT) * (d->d_inner / VEC);
+    using sambay::scan::kConvTT;
     ProfScope ps("conv_silu", st);
-    sambay::scan::conv_silu_kernel<T, TT><<<grid_for(threads, 256, sms), 256, 0, st>>>(p);
+    if (d->d_inner % 64 == 0) {
+      dim3 grid(d->d_inner / 64, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
+      sambay::scan::conv_silu_kernel<T, 64><<<grid, 64 / 4 * (kConvTT / 4), 0, st>>>(p);
+    } else {
+      dim3 grid(d->d_inner / 32, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
+      sambay::scan::conv_silu_kernel<T, 32><<<grid, 32 / 4 * (kConvTT / 4), 0, st>>>(p);
+    }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
   SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st));

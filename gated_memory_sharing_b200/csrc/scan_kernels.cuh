@@ -52,9 +52,15 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // ------------------------------------------------------- conv1d + SiLU (prefill)
 //
-// One thread: VEC consecutive channels (16 bytes of T) x TT consecutive
-// tokens, with a (K-1)-token halo taken from the previous tokens, the caller's
-// conv state (continuing prompt) or zeros (fresh prompt).
+// CTA: CB (64 or 32) consecutive channels x kConvTT (64) consecutive tokens of
+// one sequence.  The input rows t0-3 .. t0+63 of those channels land in shared
+// memory with 16-byte copies (the 3-row halo comes from the previous tokens,
+// the caller's conv state for a continuing prompt, or zeros for a fresh one),
+// so each input is read from HBM about once.  Thread: 4 consecutive channels x
+// 4 consecutive tokens, taps and bias in registers (few enough for four CTAs
+// per SM, whose loads then overlap one another's arithmetic); the outputs
+// leave as 8-byte stores (bf16: the split pair's hi row and lo row), 16
+// threads per 64-channel row.
 
 template <typename T>
 struct ConvParams {
@@ -67,20 +73,22 @@ struct ConvParams {
   int zero_init;
 };
 
-// Stores VEC conv outputs of one token row: float32 as is; bf16 as the split
+constexpr int kConvTT = 64;                   // tokens per CTA
+
+// N (4 or 8) conv outputs of one token row: float32 as is; bf16 as the split
 // pair (hi at column c, lo at column Di + c of a 2*Di row).
-template <typename T, int VEC>
-__device__ __forceinline__ void store_uc(T* uc, long long row, int Di, int c0, const float (&y)[VEC]) {
-  static_assert(VEC * sizeof(T) == 16 || VEC * sizeof(T) == 8, "16- or 8-byte vectors");
+template <typename T, int N>
+__device__ __forceinline__ void store_uc(T* uc, long long row, int Di, int c0, const float (&y)[N]) {
+  static_assert(N == 4 || N == 8, "4 or 8 outputs");
   if constexpr (sizeof(T) == 2) {
-    __nv_bfloat162 hi[VEC / 2], lo[VEC / 2];
+    __nv_bfloat162 hi[N / 2], lo[N / 2];
 #pragma unroll
-    for (int v = 0; v < VEC; v += 2) {
+    for (int v = 0; v < N; v += 2) {
       hi[v / 2] = __floats2bfloat162_rn(y[v], y[v + 1]);
       const float2 back = __bfloat1622float2(hi[v / 2]);
       lo[v / 2] = __floats2bfloat162_rn(y[v] - back.x, y[v + 1] - back.y);
     }
-    if constexpr (VEC == 8) {
+    if constexpr (N == 8) {
       *reinterpret_cast<uint4*>(uc + row * 2 * Di + c0) = *reinterpret_cast<const uint4*>(hi);
       *reinterpret_cast<uint4*>(uc + row * 2 * Di + Di + c0) = *reinterpret_cast<const uint4*>(lo);
     } else {
@@ -88,69 +96,85 @@ __device__ __forceinline__ void store_uc(T* uc, long long row, int Di, int c0, c
       *reinterpret_cast<uint2*>(uc + row * 2 * Di + Di + c0) = *reinterpret_cast<const uint2*>(lo);
     }
   } else {
-    if constexpr (VEC == 4) *reinterpret_cast<float4*>(uc + row * Di + c0) = make_float4(y[0], y[1], y[2], y[3]);
-    else *reinterpret_cast<float2*>(uc + row * Di + c0) = make_float2(y[0], y[1]);
+#pragma unroll
+    for (int v = 0; v < N; v += 4)
+      *reinterpret_cast<float4*>(uc + row * Di + c0 + v) = make_float4(y[v], y[v + 1], y[v + 2], y[v + 3]);
   }
 }
 
-template <typename T, int TT>
-__global__ void __launch_bounds__(256) conv_silu_kernel(const ConvParams<T> p) {
-  constexpr int VEC = 8 / sizeof(T);
-  const int groups = p.Di / VEC;
-  const int ttiles = (p.L + TT - 1) / TT;
-  const long long total = static_cast<long long>(p.B) * ttiles * groups;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int g = static_cast<int>(idx % groups);
-    const long long r = idx / groups;
-    const int tt = static_cast<int>(r % ttiles);
-    const int b = static_cast<int>(r / ttiles);
-    const int c0 = g * VEC;
-    const int t0 = tt * TT;
-    const long long base = static_cast<long long>(b) * p.L;
+// 4 consecutive values of T at p (8- or 16-byte aligned) as floats
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&x)[4]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  } else {
+    const float4 r = *reinterpret_cast<const float4*>(p);
+    x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+  }
+}
 
-    // rows[i] = the VEC inputs of token t0 - (K-1) + i
-    uint2 rows[TT + kK - 1];
+template <typename T, int CB>
+__global__ void __launch_bounds__(CB / 4 * (kConvTT / 4), 4) conv_silu_kernel(const ConvParams<T> p) {
+  constexpr int ROWS = kConvTT + kK - 1;
+  constexpr int EP = 16 / sizeof(T);          // elements per 16-byte piece
+  constexpr int PPR = CB / EP;                // pieces per row
+  constexpr int NT = CB / 4 * (kConvTT / 4);  // threads
+  __shared__ __align__(16) T tile[ROWS][CB];
+  const int c0 = blockIdx.x * CB;
+  const int t0 = blockIdx.y * kConvTT;
+  const int b = blockIdx.z;
+  const long long base = static_cast<long long>(b) * p.L;
+
+  for (int i = threadIdx.x; i < ROWS * PPR; i += NT) {
+    const int r = i / PPR, piece = i % PPR;
+    const int t = t0 - (kK - 1) + r;
+    T* d = &tile[r][piece * EP];
+    if (t >= 0 && t < p.L) {
+      cp_async16(d, p.u + (base + t) * p.Di + c0 + piece * EP);
+    } else if (t < 0 && !p.zero_init) {
+      // left context: entry K + t of each channel's conv state
 #pragma unroll
-    for (int i = 0; i < TT + kK - 1; ++i) {
-      const int t = t0 - (kK - 1) + i;
-      rows[i] = make_uint2(0u, 0u);
-      if (t >= 0 && t < p.L) rows[i] = *reinterpret_cast<const uint2*>(p.u + (base + t) * p.Di + c0);
+      for (int e = 0; e < EP; ++e)
+        d[e] = p.conv_state[(static_cast<long long>(b) * p.Di + c0 + piece * EP + e) * kK + kK + t];
+    } else {
+      *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (t0 == 0 && !p.zero_init) {
-      // left context from the conv state: entry K + t of each channel for t < 0
+  }
+  cp_async_commit();
+
+  const int j = threadIdx.x % (CB / 4);       // channels c0 + 4j .. + 3
+  const int tq = threadIdx.x / (CB / 4);      // tokens t0 + 4tq .. + 3
+  const int cj = c0 + 4 * j;
+  float w[4][kK], bias[4];
+  {
+    // 4 channels x K taps are 4K contiguous values
 #pragma unroll
-      for (int i = 0; i < kK - 1; ++i) {
-        T* e = reinterpret_cast<T*>(&rows[i]);
+    for (int v = 0; v < 4; ++v) load4<T>(p.conv_w + static_cast<long long>(cj + v) * kK, w[v]);
+    load4<T>(p.conv_b + cj, bias);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // output token t0 + 4tq + i reads tile rows 4tq + i .. 4tq + i + K - 1
+  // (tile row r is token t0 - K + 1 + r)
 #pragma unroll
-        for (int v = 0; v < VEC; ++v)
-          e[v] = p.conv_state[(static_cast<long long>(b) * p.Di + c0 + v) * kK + 1 + i];
-      }
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + 4 * tq + i;
+    if (t >= p.L) break;
+    float y[4] = {bias[0], bias[1], bias[2], bias[3]};
+#pragma unroll
+    for (int k = 0; k < kK; ++k) {
+      float x[4];
+      load4<T>(&tile[4 * tq + i + k][4 * j], x);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) y[v] = fmaf(w[v][k], x[v], y[v]);
     }
-    // taps in registers: the uc stores below could alias them as far as the
-    // compiler knows, so loads inside the token loop would be repeated
-    float w[VEC][kK], bias[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-      bias[v] = to_f32(p.conv_b[c0 + v]);
-#pragma unroll
-      for (int k = 0; k < kK; ++k) w[v][k] = to_f32(p.conv_w[(c0 + v) * kK + k]);
-    }
-#pragma unroll
-    for (int i = 0; i < TT; ++i) {
-      const int t = t0 + i;
-      if (t >= p.L) break;
-      float y[VEC];
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        float acc = bias[v];
-#pragma unroll
-        for (int k = 0; k < kK; ++k)
-          acc = fmaf(w[v][k], to_f32(reinterpret_cast<const T*>(&rows[i + k])[v]), acc);
-        y[v] = silu(acc);
-      }
-      store_uc<T, VEC>(p.uc, base + t, p.Di, c0, y);
-    }
+    for (int v = 0; v < 4; ++v) y[v] = silu(y[v]);
+    store_uc<T, 4>(p.uc, base + t, p.Di, cj, y);
   }
 }
 
