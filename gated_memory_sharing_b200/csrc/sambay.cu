@@ -481,7 +481,7 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     if (rows <= sambay::tc::BM)   // one row tile (decode): narrower tiles, more CTAs
       SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
     else
-      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
+      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st, true)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
     SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
