@@ -186,8 +186,7 @@ ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
 }
 
 struct GmuWs {
-  size_t h, part, counters, total;
-  int splits1, splits2;
+  size_t h, part, total;
 };
 
 constexpr int kStepMaxRows = 256;
@@ -199,15 +198,10 @@ GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
   w.h = off;
   off += round256(static_cast<size_t>(rows) * d->d_inner * io_bytes(d->io));
   if (step && d->io == SAMBAY_BF16) {
-    // swap-AB: output tiles run over d_inner (GEMM1) and d_model (GEMM2)
-    w.splits1 = split_count((d->d_inner + 127) / 128, d->d_model, kStepMaxSplits);
-    w.splits2 = split_count((d->d_model + 127) / 128, d->d_inner, kStepMaxSplits);
+    // swap-AB split-K partials, room for kStepMaxSplits splits of either GEMM
+    // (output tiles over d_inner for GEMM1, d_model for GEMM2)
     w.part = off;
-    off += round256(static_cast<size_t>(rows) *
-                    std::max(static_cast<long long>(w.splits1) * d->d_inner,
-                             static_cast<long long>(w.splits2) * d->d_model) * 4);
-    w.counters = off;
-    off += round256(static_cast<size_t>((d->d_inner + 127) / 128 + (d->d_model + 127) / 128) * 4);
+    off += round256(static_cast<size_t>(rows) * kStepMaxSplits * std::max(d->d_inner, d->d_model) * 4);
   }
   w.total = off;
   return w;
@@ -284,6 +278,34 @@ TailPlan tail_plan(int tiles, int BN, int slots, int min_width) {
   return tp;
 }
 
+// Whether `count` clusters of `s` CTAs of this (non-pair) configuration are
+// co-resident on the device; cached per device and cluster size.
+template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW>
+bool cluster_fits(int dev, int sms, int s, int count) {
+  using namespace sambay::tc;
+  using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, false>;
+  static int active[kMaxDevices][9] = {};
+  if (active[dev][s] == 0) {
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(s * (sms / s));
+    q.blockDim = dim3(gemm_threads(EW));
+    q.dynamicSmemBytes = C::kSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = s;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    q.attrs = at;
+    q.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS, EW, false>, &q) !=
+            cudaSuccess)
+      n = -1;
+    active[dev][s] = n > 0 ? n : -1;
+  }
+  return active[dev][s] >= count;
+}
+
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
 // split_count for the same sizes); `balance_tail` (no K split) applies
 // tail_plan.  PAIR: 256-row tiles on CTA pairs (clusters of two).
@@ -344,9 +366,22 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   g.m_tiles = (g.M + C::kBMT - 1) / C::kBMT;
   g.n_tiles = (g.N + BN - 1) / BN;
   g.k_blocks = (g.K + BK - 1) / BK;
+  if (g.csplit) {
+    // cluster split-K: the most splits (<= `splits`) whose clusters of that
+    // many CTAs all fit on the GPU at once, about one CTA per SM in total
+    const int tiles = g.m_tiles * g.n_tiles;
+    int best = 1;
+    for (int s = std::min({splits, g.k_blocks, 8}); s >= 2; --s) {
+      if (static_cast<long long>(tiles) * s > sms) continue;
+      if (cluster_fits<BN, A_MN, B_MN, KIND, TRANS, EW>(dev, sms, s, tiles)) { best = s; break; }
+    }
+    splits = best;
+    if (splits == 1) g.csplit = 0;
+  }
   splits = std::max(1, std::min(splits, g.k_blocks));
   g.kb_per_split = (g.k_blocks + splits - 1) / splits;
   g.splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
+  if (g.splits == 1) g.csplit = 0;
   g.tiles = g.m_tiles * g.n_tiles * g.splits;
   g.full_tiles = g.tiles;
   g.tail_nsplit = 1;
@@ -376,6 +411,21 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
       cudaLaunchAttribute at[1];
       at[0].id = cudaLaunchAttributeClusterDimension;
       at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      lc.attrs = at;
+      lc.numAttrs = 1;
+      if (cudaLaunchKernelEx(&lc, kern, ta, tb, tb2, taux, tout, g) != cudaSuccess) return SAMBAY_ERR_CUDA;
+    } else if (g.csplit) {
+      // one unit per CTA; the splits of a tile are one cluster
+      cudaLaunchConfig_t lc = {};
+      lc.gridDim = dim3(g.tiles);
+      lc.blockDim = dim3(gemm_threads(EW));
+      lc.dynamicSmemBytes = C::kSmem;
+      lc.stream = st;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = g.splits;
       at[0].val.clusterDim.y = 1;
       at[0].val.clusterDim.z = 1;
       lc.attrs = at;
@@ -771,17 +821,16 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   const int Dm = d->d_model, Di = d->d_inner, Bn = static_cast<int>(rows);
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   float* part = reinterpret_cast<float*>(w8 + L.part);
-  int* counters = reinterpret_cast<int*>(w8 + L.counters);
-  // split-K arrival counters start at zero; the last CTA of each tile resets
-  // its counter, so the second GEMM finds them zero again
-  if (cudaMemsetAsync(counters, 0, L.total - L.counters, st) != cudaSuccess) return SAMBAY_ERR_CUDA;
-  // swap-AB: H^T = SiLU(W1 X^T) ⊙ M^T; W1 rows stream once through the tensor cores
-  const auto g1 = tc_args(Di, Bn, Dm, H, Di, M, nullptr, part, rows * static_cast<long long>(Di), counters);
-  const auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual, nullptr, part, rows * static_cast<long long>(Dm), counters);
+  // swap-AB: H^T = SiLU(W1 X^T) ⊙ M^T; W1 rows stream once through the tensor
+  // cores.  Split-K over clusters of CTAs (csplit): the splits of a tile meet
+  // at a cluster barrier and each finishes a slice of its rows.
+  auto g1 = tc_args(Di, Bn, Dm, H, Di, M, nullptr, part, rows * static_cast<long long>(Di));
+  auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual, nullptr, part, rows * static_cast<long long>(Dm));
+  g1.csplit = g2.csplit = 1;
   const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
 #define SAMBAY_STEP_GEMMS(BNV)                                                                   \
-  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, L.splits1, st))); \
-  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, L.splits2, st)));
+  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, kStepMaxSplits, st))); \
+  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, kStepMaxSplits, st)));
   if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
   else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
   else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }

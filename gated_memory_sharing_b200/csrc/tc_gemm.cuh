@@ -304,6 +304,11 @@ struct GemmArgs {
   int tma_epi;        // row-major gate / residual / softplus epilogue through TMA
                       // (aux tile in, output tile out); set by the host when the
                       // output's columns come in whole 64 (bf16) / 32 (f32) blocks
+  int csplit;         // cluster split-K: the `splits` K ranges of a tile are one
+                      // cluster of CTAs (one unit each), which write their partial
+                      // tiles, meet at a cluster barrier and then each reduce and
+                      // finish a slice of the tile's rows (no counters, no tail
+                      // where one CTA sums every partial)
   int full_tiles;     // tail_nsplit > 1: work units [0, full_tiles) are whole tiles,
   int tail_nsplit;    // and every later tile is cut along N into tail_nsplit units
                       // of BN / tail_nsplit columns (wave quantisation: the last,
@@ -500,10 +505,17 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
     c.kb1 = g.k_blocks;
     return c;
   }
-  c.m = t % g.m_tiles;
-  const int r = t / g.m_tiles;
-  c.n = r % g.n_tiles;
-  c.split = r / g.n_tiles;
+  if (g.csplit) {             // unit t: split t % splits of tile t / splits
+    c.split = t % g.splits;
+    const int tile = t / g.splits;
+    c.m = tile % g.m_tiles;
+    c.n = tile / g.m_tiles;
+  } else {
+    c.m = t % g.m_tiles;
+    const int r = t / g.m_tiles;
+    c.n = r % g.n_tiles;
+    c.split = r / g.n_tiles;
+  }
   c.kb0 = c.split * g.kb_per_split;
   c.kb1 = min(g.k_blocks, c.kb0 + g.kb_per_split);
   c.n0 = c.n * BN;
@@ -868,7 +880,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
-      if (split) {
+      if (split && !g.csplit) {
         // The last CTA to finish a split-K tile sums the partials in split
         // order (deterministic), applies the final op and resets the counter.
         __threadfence();
@@ -919,6 +931,29 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
   if (PAIR) cluster_sync();
   else __syncthreads();
   tc_fence_after();
+  if (!PAIR && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {
+    // cluster split-K: every CTA of the cluster has written its partial tile;
+    // CTA `split` now sums rows [split * R, +R) of the tile over the splits in
+    // split order and applies the final op
+    __threadfence();
+    cluster_sync();
+    const TileCoord c = tile_coord<BN>(g, blockIdx.x);
+    const int R = (BM + g.splits - 1) / g.splits;
+    const int r0 = c.split * R, r1 = min(BM, r0 + R);
+    const int nrows = max(0, r1 - r0), ncols = min(c.bn, g.N - c.n0);
+    for (int e = threadIdx.x; e < nrows * ncols; e += blockDim.x) {
+      const int m = c.m * BM + r0 + e % nrows;   // consecutive threads: consecutive rows
+      const int n = c.n0 + e / nrows;
+      if (m >= g.M) continue;
+      const long long o = TRANS ? static_cast<long long>(n) * g.ldo + m : static_cast<long long>(m) * g.ldo + n;
+      float v = 0.0f;
+      for (int sp = 0; sp < g.splits; ++sp) v += __ldcg(g.partials + static_cast<long long>(sp) * g.split_stride + o);
+      float a = 0.0f;
+      if (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr))
+        a = to_f32(reinterpret_cast<const bf16*>(g.aux)[o]);
+      epi_store_one<KIND>(g, o, n, v, a);
+    }
+  }
   if (warp == 1) {
     if (PAIR)
       asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
