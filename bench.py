@@ -37,7 +37,16 @@ WORKLOAD = "prefill_b1_l2048"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
 # kernel, from one ncu capture of the benchmarked workload (profiles/); a kernel
 # changed since its capture has no entry (reported as null).
-DRAM_TRAFFIC = {}
+DRAM_TRAFFIC = {
+    # profiles/prefill_b1_l2048_launches.md (bench.py --steps 3 --warmup 3 --no-cpu-baseline --no-decode)
+    "conv_silu": 21034240 + 86016,
+    "x_proj": 43944448 + 768,
+    "xdbl_reduce": 14177280 + 0,
+    "dt_proj": 3315712 + 0,
+    "selective_scan": 84559872 + 2316288,
+    "gmu_gate_gemm": 57750784 + 175872,
+    "gmu_out_gemm": 47247360 + 77824,
+}
 METRIC = "scan+GMU prefill tokens/s"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
