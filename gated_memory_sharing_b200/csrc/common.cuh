@@ -61,6 +61,20 @@ __device__ __forceinline__ float softplus(float x) {
   return fmaxf(x, 0.0f) + (y < 0.0625f ? series : viaLog);
 }
 
+// 16-byte load through L2 (no L1 allocation) of p when `pred`, else zeros.
+// Written as a predicated load rather than a branch so a run of these stays
+// independent and the compiler keeps them all in flight at once.
+__device__ __forceinline__ float4 ldcg_or_zero(const float* p, bool pred) {
+  float4 v;
+  asm("{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+      "@q ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];\n\t}"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+      : "l"(p), "r"(static_cast<int>(pred)));
+  return v;
+}
+
 // Pack / unpack helpers for 16-byte vector access.
 union Pack16 {
   uint4 u;

@@ -186,11 +186,14 @@ ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
 }
 
 struct GmuWs {
-  size_t h, part, total;
+  size_t h, part, tail, tail_bytes, total;
 };
 
 constexpr int kStepMaxRows = 256;
 constexpr int kStepMaxSplits = 8;
+// Partial tiles of a prefill GEMM's K-split tail: at most one 256 x 256 fp32
+// tile per CTA pair of a 148-SM B200.
+constexpr int kTailUnits = 74;
 
 GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
   GmuWs w{};
@@ -202,6 +205,12 @@ GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
     // (output tiles over d_inner for GEMM1, d_model for GEMM2)
     w.part = off;
     off += round256(static_cast<size_t>(rows) * kStepMaxSplits * std::max(d->d_inner, d->d_model) * 4);
+  }
+  if (!step && d->io == SAMBAY_BF16 && rows > 256) {
+    // more than one 256-row tile: room for the K-split tail of either GEMM
+    w.tail = off;
+    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4;
+    off += round256(w.tail_bytes);
   }
   w.total = off;
   return w;
@@ -257,6 +266,29 @@ struct Operand {
   long long rows, cols;
 };
 
+// The kernels launched between the tensor-core GEMMs ask for the largest
+// shared-memory carveout, the configuration the GEMMs need, so the SMs keep
+// one L1 / shared-memory split through a whole step instead of switching it
+// at kernel boundaries.  Once per call site (kernel) and device; a refusal
+// only leaves the default preference.
+#define SAMBAY_MAX_CARVEOUT(kern, dev)                                                  \
+  do {                                                                                  \
+    static bool done_[kMaxDevices] = {};                                                \
+    if (!done_[dev]) {                                                                  \
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,    \
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess)          \
+        (void)cudaGetLastError();                                                       \
+      done_[dev] = true;                                                                \
+    }                                                                                   \
+  } while (0)
+
+// Blocks for a grid-stride launch of `threads` threads: enough to cover
+// them, at most 16 per SM.
+int grid_for(long long threads, int block, int sms) {
+  const long long g = (threads + block - 1) / block;
+  return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(sms) * 16)));
+}
+
 // Last-wave balancing of a GEMM without K split: with W whole waves of
 // tiles over the SMs and a partial wave of `tail` tiles, the tail tiles are
 // cut along N into nsplit units (64 columns at the narrowest) so they spread
@@ -276,6 +308,26 @@ TailPlan tail_plan(int tiles, int BN, int slots, int min_width) {
       break;
     }
   return tp;
+}
+
+// K-split tail (pairs only): the partial wave's `ntail` tiles are each cut
+// along K into `splits` units of `kbps` k-blocks (ntail * splits <= slots);
+// every unit writes an fp32 partial tile and tail_reduce_kernel sums them in
+// split order and applies the epilogue.
+struct KTailPlan {
+  int ntail = 0, splits = 1, kbps = 0;
+};
+
+KTailPlan ktail_plan(int tiles, int slots, int k_blocks) {
+  KTailPlan kp;
+  const int waves = tiles / slots, tail = tiles % slots;
+  if (waves == 0 || tail == 0) return kp;
+  const int s = std::min({slots / tail, k_blocks, sambay::tc::kMaxTailSplits});
+  if (s < 2) return kp;
+  kp.kbps = (k_blocks + s - 1) / s;
+  kp.splits = (k_blocks + kp.kbps - 1) / kp.kbps;
+  if (kp.splits >= 2) kp.ntail = tail;
+  return kp;
 }
 
 // Whether `count` clusters of `s` CTAs of this (non-pair) configuration are
@@ -308,15 +360,21 @@ bool cluster_fits(int dev, int sms, int s, int count) {
 
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
 // split_count for the same sizes); `balance_tail` (no K split) applies
-// tail_plan.  PAIR: 256-row tiles on CTA pairs (clusters of two).
+// tail_plan, or for pairs with `tail_part` scratch of `tail_bytes` the
+// K-split tail when that leaves the shorter last round (a tail unit costs
+// 1/splits of a tile plus about a tenth of one for its partial tile and the
+// reduction, launched as `tail_name`).  PAIR: 256-row tiles on CTA pairs
+// (clusters of two).
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4, bool PAIR = false>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
-                     sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false) {
+                     sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false,
+                     float* tail_part = nullptr, size_t tail_bytes = 0, const char* tail_name = nullptr) {
   using namespace sambay::tc;
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   static bool attr_set[kMaxDevices] = {};
   static int pair_slots[kMaxDevices] = {};   // co-resident clusters of two (PAIR)
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
+  SAMBAY_MAX_CARVEOUT(kern, dev);
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem)) != cudaSuccess)
@@ -386,12 +444,24 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   g.full_tiles = g.tiles;
   g.tail_nsplit = 1;
   CUtensorMap tb2 = tb;
+  g.tail_ksplit = 1;
   const int slots = PAIR ? pair_slots[dev] : sms;   // work units in flight at once
+  int ktail = 0;
   if (balance_tail && g.splits == 1) {
     // narrowest unit: 64 columns per CTA's B load (MN-major B: whole 64-column boxes)
     const int min_width = (PAIR && B_MN) ? 128 : 64;
     const TailPlan tp = tail_plan(g.tiles, BN, slots, min_width);
-    if (tp.nsplit > 1) {
+    const KTailPlan kp = PAIR && tail_part ? ktail_plan(g.tiles, slots, g.k_blocks) : KTailPlan{};
+    const double ncost = 1.0 / tp.nsplit, kcost = 1.0 / kp.splits + 0.1;
+    if (kp.ntail > 0 && kcost < ncost &&
+        static_cast<size_t>(kp.ntail) * kp.splits * C::kBMT * BN * 4 <= tail_bytes) {
+      g.full_tiles = g.tiles - kp.ntail;
+      g.tail_ksplit = kp.splits;
+      g.tail_kbps = kp.kbps;
+      g.tail_part = tail_part;
+      g.tiles = g.full_tiles + kp.ntail * kp.splits;
+      ktail = kp.ntail;
+    } else if (tp.nsplit > 1) {
       const int hb = (BN / tp.nsplit) / (PAIR ? 2 : 1);
       if (!B_MN && !make_map(&tb2, b.ptr, b.cols, b.rows, b.cols * 2, hb)) return SAMBAY_ERR_CUDA;
       g.tiles = tp.full + (g.tiles - tp.full) * tp.nsplit;
@@ -434,6 +504,14 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
     } else {
       kern<<<units, gemm_threads(EW), C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
     }
+  }
+  if constexpr (PAIR) if (ktail > 0) {
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+    const long long work = static_cast<long long>(ktail) * C::kBMT * (BN / 4) * kTailLanes;
+    auto rk = tail_reduce_kernel<BN, C::kBMT, KIND>;
+    SAMBAY_MAX_CARVEOUT(rk, dev);
+    ProfScope ps(tail_name ? tail_name : "gemm_tail_reduce", st);
+    rk<<<grid_for(work, 256, sms), 256, 0, st>>>(g, ktail);
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -482,11 +560,6 @@ sambay::simt::Args simt_args(const float* A, long long sam, long long sak, const
     if (_s != SAMBAY_OK) return _s;      \
   } while (0)
 
-int grid_for(long long threads, int block, int sms) {
-  const long long g = (threads + block - 1) / block;
-  return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(sms) * 16)));
-}
-
 // ------------------------------------------------------------ shared scan pieces
 
 // x_proj + dt_proj for `rows` tokens whose conv output is ws.uc:
@@ -514,13 +587,16 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
     else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
     {
+      auto k8 = sambay::scan::xdbl_reduce_kernel<8>;
+      auto k1 = sambay::scan::xdbl_reduce_kernel<1>;
+      SAMBAY_MAX_CARVEOUT(k8, dev);
+      SAMBAY_MAX_CARVEOUT(k1, dev);
+      const int Lseq = static_cast<int>(rows / d->batch), nrows = static_cast<int>(rows);
       ProfScope ps_reduce("xdbl_reduce", st);
       if (L.splits >= 16)
-        sambay::scan::xdbl_reduce_kernel<8><<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(
-            part, L.splits, stride, xdbl, delta, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, Rp, ldx);
+        k8<<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx);
       else
-        sambay::scan::xdbl_reduce_kernel<1><<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(
-            part, L.splits, stride, xdbl, delta, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, Rp, ldx);
+        k1<<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx);
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
@@ -584,6 +660,7 @@ sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cuda
       return SAMBAY_ERR_CUDA;
     attr_set[dev] = true;
   }
+  SAMBAY_MAX_CARVEOUT(kern, dev);
   scan_partition<T>(p, sms);
   const ScanLayout ly(p.chp, sizeof(T));
   dim3 grid(p.nblk, p.B);
@@ -605,13 +682,17 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
                                   static_cast<const T*>(w->conv_b), uc, d->batch, d->seqlen,
                                   d->d_inner, zero_init};
     using sambay::scan::kConvTT;
+    auto c64 = sambay::scan::conv_silu_kernel<T, 64>;
+    auto c32 = sambay::scan::conv_silu_kernel<T, 32>;
+    SAMBAY_MAX_CARVEOUT(c64, dev);
+    SAMBAY_MAX_CARVEOUT(c32, dev);
     ProfScope ps("conv_silu", st);
     if (d->d_inner % 64 == 0) {
       dim3 grid(d->d_inner / 64, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
-      sambay::scan::conv_silu_kernel<T, 64><<<grid, 64 / 4 * (kConvTT / 4), 0, st>>>(p);
+      c64<<<grid, 64 / 4 * (kConvTT / 4), 0, st>>>(p);
     } else {
       dim3 grid(d->d_inner / 32, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
-      sambay::scan::conv_silu_kernel<T, 32><<<grid, 32 / 4 * (kConvTT / 4), 0, st>>>(p);
+      c32<<<grid, 32 / 4 * (kConvTT / 4), 0, st>>>(p);
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
@@ -645,16 +726,20 @@ sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, con
   const ScanWs L = scan_ws_layout(d, B);
   T* uc = reinterpret_cast<T*>(ws + L.uc);
   constexpr int VEC = 16 / sizeof(T);
+  auto sc = sambay::scan::step_conv_kernel<T>;
+  auto ss = sambay::scan::step_scan_kernel<T>;
+  SAMBAY_MAX_CARVEOUT(sc, dev);
+  SAMBAY_MAX_CARVEOUT(ss, dev);
   {
     ProfScope ps("step_conv", st);
-    sambay::scan::step_conv_kernel<T><<<grid_for(B * (d->d_inner / VEC), 256, 1 << 20), 256, 0, st>>>(
+    sc<<<grid_for(B * (d->d_inner / VEC), 256, 1 << 20), 256, 0, st>>>(
       static_cast<const T*>(u_t), static_cast<T*>(conv_state), static_cast<const T*>(w->conv_w),
       static_cast<const T*>(w->conv_b), uc, d->batch, d->d_inner);
   }
   if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st));
   ProfScope ps("step_scan", st);
-  sambay::scan::step_scan_kernel<T><<<grid_for(B * d->d_inner * 4, 256, 1 << 20), 256, 0, st>>>(
+  ss<<<grid_for(B * d->d_inner * 4, 256, 1 << 20), 256, 0, st>>>(
       uc, reinterpret_cast<const float*>(ws + L.dt), reinterpret_cast<const float*>(ws + L.xdbl),
       w->A, w->D, ssm_state, static_cast<T*>(m_t), d->batch, d->d_inner, d->dt_rank,
       d->dt_rank + 2 * d->d_state);
@@ -796,13 +881,15 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, residual, Y, w8, L, st);
   const int Dm = d->d_model, Di = d->d_inner, T = static_cast<int>(rows);
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
+  float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8, true>(
-      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true)));
+      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true,
+      tail, L.tail_bytes, "gmu_gate_tail")));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
   SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8, true>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
-      st, true)));
+      st, true, tail, L.tail_bytes, "gmu_out_tail")));
   return SAMBAY_OK;
 }
 

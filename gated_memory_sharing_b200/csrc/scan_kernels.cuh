@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(CB / 4 * (kConvTT / 4), 4) conv_silu_kernel(co
 // LPG lanes per 4-column group: lane `sub` adds splits sub, sub + LPG, ... in
 // order, then a fixed xor tree combines the lane sums, so the result is the
 // same on every run.  Warps iterate uniformly (shuffles need all lanes).
-// LPG = 8 for many splits (single-row-tile decode), 1 otherwise.
+// LPG = 8 for 16 or more splits (single-row-tile decode), 1 otherwise.
 template <int LPG>
 __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int splits,
                                    long long split_stride, float* __restrict__ xdbl,
@@ -205,10 +205,19 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
     const bool valid = i < total4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (valid) {
-#pragma unroll 4
-      for (int sp = sub; sp < splits; sp += LPG) {
-        const float4 p = reinterpret_cast<const float4*>(partials + sp * split_stride)[i];
-        acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+      // a batch of this lane's splits loaded together, then added in order
+#pragma unroll 1
+      for (int s0 = sub; s0 < splits; s0 += 4 * LPG) {
+        float4 p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int sp = s0 + j * LPG;
+          p[j] = ldcg_or_zero(partials + (sp < splits ? sp * split_stride + 4 * i : 0), sp < splits);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc.x += p[j].x; acc.y += p[j].y; acc.z += p[j].z; acc.w += p[j].w;
+        }
       }
     }
 #pragma unroll

@@ -313,6 +313,10 @@ struct GemmArgs {
   int tail_nsplit;    // and every later tile is cut along N into tail_nsplit units
                       // of BN / tail_nsplit columns (wave quantisation: the last,
                       // partial wave of tiles spreads over more SMs; no K split)
+  int tail_ksplit;    // > 1 instead: every tile after full_tiles is cut along K into
+  int tail_kbps;      // tail_ksplit units of tail_kbps k-blocks, each writing its fp32
+  float* tail_part;   // partial tile [tail tile][split][tile rows][BN] to tail_part;
+                      // tail_reduce_kernel sums them and applies the epilogue
 };
 
 // The final op on one element.  `o` is the output's linear index, `a` the aux
@@ -488,11 +492,26 @@ struct Cfg {
 struct TileCoord {
   int m, n, split, kb0, kb1;
   int n0, bn;          // first output column and width of this unit
+  int tailk;           // -1, or the index among the K-split tail tiles
 };
 
 template <int BN>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   TileCoord c;
+  c.tailk = -1;
+  if (g.tail_ksplit > 1 && t >= g.full_tiles) {
+    const int r = t - g.full_tiles;
+    c.tailk = r / g.tail_ksplit;
+    const int tile = g.full_tiles + c.tailk;
+    c.m = tile % g.m_tiles;
+    c.n = tile / g.m_tiles;
+    c.bn = BN;
+    c.n0 = c.n * BN;
+    c.split = r % g.tail_ksplit;
+    c.kb0 = c.split * g.tail_kbps;
+    c.kb1 = min(g.k_blocks, c.kb0 + g.tail_kbps);
+    return c;
+  }
   if (g.tail_nsplit > 1 && t >= g.full_tiles) {
     const int r = t - g.full_tiles;
     const int tile = g.full_tiles + r / g.tail_nsplit;
@@ -710,7 +729,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     for (int t = unit0; t < g.tiles; t += ustride) {
       const TileCoord c = tile_coord<BN>(g, t);
       const int arow = c.m * C::kBMT + rank * BM;     // this CTA's first output row
-      const bool split = g.splits > 1 && KIND != EPI_F32_PARTIAL;
+      const bool split = (g.splits > 1 && KIND != EPI_F32_PARTIAL) || c.tailk >= 0;
       const bool tma = C::kTmaEpi && g.tma_epi && !split;
       if (tma) {
         // the tile's aux blocks (M or the residual) and bias are fetched while
@@ -850,7 +869,15 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
         const int n0 = c.n0 + ch * 32;
-        if (split) {
+        if (c.tailk >= 0) {
+          // K-split tail unit: this CTA's rows of the partial tile, row-major
+          float* part = g.tail_part +
+                        ((static_cast<long long>(c.tailk) * g.tail_ksplit + c.split) * C::kBMT +
+                         (row - c.m * C::kBMT)) * BN + (n0 - c.n0);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            __stcg(reinterpret_cast<float4*>(part + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+        } else if (split) {
           // this split's partial tile, summed in split order by the last CTA
           float* part = g.partials + static_cast<long long>(c.split) * g.split_stride;
           if (row < g.M) {
@@ -880,7 +907,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
 
-      if (split && !g.csplit) {
+      if (split && !g.csplit && c.tailk < 0) {
         // The last CTA to finish a split-K tile sums the partials in split
         // order (deterministic), applies the final op and resets the counter.
         __threadfence();
@@ -963,6 +990,64 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                    "r"(C::kTmemCols)
                    : "memory");
+  }
+}
+
+// The K-split tail tiles of a GEMM: out = epilogue(sum of the tail_ksplit
+// (<= kMaxTailSplits) partial tiles).  kTailLanes lanes share one output
+// float4 (4 consecutive columns of a row): lane `sub` adds splits sub,
+// sub + kTailLanes, ... in order, then a fixed xor tree combines the lanes,
+// so the result is the same on every run.  Warps iterate uniformly (shuffles
+// need all lanes).
+constexpr int kMaxTailSplits = 16;
+constexpr int kTailLanes = 4;
+
+template <int BN, int BMT, int KIND>
+__global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmArgs g, int ntail) {
+  constexpr int Q = BN / 4, LPG = kTailLanes, PER = kMaxTailSplits / LPG;
+  const int lane = threadIdx.x & 31, sub = lane % LPG;
+  const long long total = static_cast<long long>(ntail) * BMT * Q;   // output float4s
+  const long long warps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
+  for (long long w = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
+       w * (32 / LPG) < total; w += warps) {
+    const long long e = w * (32 / LPG) + lane / LPG;
+    const int i = static_cast<int>(e / (BMT * Q));
+    const int lr = static_cast<int>((e / Q) % BMT), lq = static_cast<int>(e % Q);
+    const int tile = g.full_tiles + i;
+    const int m = (tile % g.m_tiles) * BMT + lr;
+    const int n = (tile / g.m_tiles) * BN + 4 * lq;
+    const bool live = e < total && m < g.M && n < g.N;
+    const float* base = g.tail_part + (static_cast<long long>(i) * g.tail_ksplit * BMT + lr) * BN + 4 * lq;
+    float4 x[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int sp = sub + j * LPG;
+      const bool on = live && sp < g.tail_ksplit;
+      x[j] = ldcg_or_zero(base + (on ? static_cast<long long>(sp) * BMT * BN : 0), on);
+    }
+    float4 acc = x[0];
+#pragma unroll
+    for (int j = 1; j < PER; ++j) {
+      acc.x += x[j].x; acc.y += x[j].y; acc.z += x[j].z; acc.w += x[j].w;
+    }
+#pragma unroll
+    for (int off = LPG / 2; off >= 1; off >>= 1) {
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+    }
+    if (!live || sub != 0) continue;
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    const long long o = static_cast<long long>(m) * g.ldo + n;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (n + j >= g.N) break;
+      float a = 0.0f;
+      if (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr))
+        a = to_f32(reinterpret_cast<const bf16*>(g.aux)[o + j]);
+      epi_store_one<KIND>(g, o + j, n + j, v[j], a);
+    }
   }
 }
 

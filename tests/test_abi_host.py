@@ -70,7 +70,10 @@ def test_workspace_queries(lib):
     f = abi.make_dims(1, 64, 64, 128, 16, 4, 4, abi.F32)
     assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4) \
         + r256(32 * 64 * 4)
-    assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2)
+    # H, then (more than one 256-row tile) one fp32 256 x 256 partial tile per
+    # CTA pair of 148 SMs for a GEMM's K-split tail
+    assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2) + r256(74 * 256 * 256 * 4)
+    assert abi.gmu_forward_workspace(d, 256) == r256(256 * 5120 * 2)
     assert abi.gmu_step_workspace(d, 64) > 64 * 5120 * 2
     # invalid or unsupported dims -> 0
     assert abi.sambay_scan_prefill_workspace(abi.make_dims(1, 16, 64, 128, 8, 4, 8, abi.BF16)) == 0

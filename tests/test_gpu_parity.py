@@ -75,6 +75,26 @@ def test_gmu_forward_multi_tile_bf16():
     assert_close(host(Y), Yr, TOL_BF16, "gmu_forward multi-tile")
 
 
+@pytest.mark.parametrize("rows,d_model,d_inner", [
+    (1900, 2560, 1024),     # GEMM2: 8 x 10 tiles of 256 x 256 on 74 CTA pairs, the last 6 cut along K
+    (500, 768, 12032),      # GEMM1: 2 x 47 tiles, the last 20 cut along K into 3
+])
+def test_gmu_forward_k_split_tail_bf16(rows, d_model, d_inner):
+    # more 256-row tiles than CTA pairs: the partial last round runs as K
+    # ranges whose fp32 partial tiles a second kernel sums in split order
+    d = synth.Dims(1, 1, d_model, d_inner, 16, 4, 16, synth.BF16)
+    seed = 15
+    gw = synth.gmu_weights(d, seed)
+    X = synth.gmu_inputs(d, seed, rows=rows)
+    M = synth.memory_input(d, seed, rows=rows)
+    g = GMULayer(gw["W1"], gw["W2"], abi.BF16)
+    Y = g.forward(to_device(X, abi.BF16), to_device(M, abi.BF16), residual=True)
+    Yr, _, _ = ref.gmu_ref(X, M, gw["W1"], gw["W2"], residual=True)
+    assert_close(host(Y), Yr, TOL_BF16, f"gmu_forward K-split tail rows={rows}")
+    # deterministic: the same bits on a second call
+    assert torch.equal(Y, g.forward(to_device(X, abi.BF16), to_device(M, abi.BF16), residual=True))
+
+
 def test_gmu_forward_in_place_residual_bf16():
     d = SMALL["bf16"]
     seed = 13
