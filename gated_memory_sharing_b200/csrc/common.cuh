@@ -61,6 +61,18 @@ __device__ __forceinline__ float softplus(float x) {
   return fmaxf(x, 0.0f) + (y < 0.0625f ? series : viaLog);
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running; pdl_wait() returns once that kernel has finished and its writes are
+// visible, so every global access that can depend on it comes after the wait.
+// pdl_launch_dependents() lets the next such kernel start launching (its CTAs
+// then sit in their own pdl_wait until this grid has finished).  Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 16-byte load through L2 (no L1 allocation) of p when `pred`, else zeros.
 // Written as a predicated load rather than a branch so a run of these stays
 // independent and the compiler keeps them all in flight at once.

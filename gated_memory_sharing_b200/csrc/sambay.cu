@@ -282,6 +282,40 @@ struct Operand {
     }                                                                                   \
   } while (0)
 
+// Kernel launch with an optional cluster size and, for `chained` launches,
+// programmatic dependent launch: used for every kernel of an entry point
+// after its first, whose predecessor on the stream is then one of this
+// library's kernels.  Such a kernel may start (set-up, CTA launch) while its
+// predecessor finishes; each kernel waits for its predecessor (pdl_wait)
+// before touching global memory.  The first kernel of a call is launched
+// plainly and so orders after whatever the caller queued before.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool chained, int cluster, Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute at[2];
+  unsigned n = 0;
+  if (cluster > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = cluster;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (chained) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  lc.attrs = at;
+  lc.numAttrs = n;
+  return cudaLaunchKernelEx(&lc, kern, args...);
+}
+
 // Blocks for a grid-stride launch of `threads` threads: enough to cover
 // them, at most 16 per SM.
 int grid_for(long long threads, int block, int sms) {
@@ -359,7 +393,9 @@ bool cluster_fits(int dev, int sms, int s, int count) {
 }
 
 // `splits` > 1 splits K into that many contiguous ranges (as computed by
-// split_count for the same sizes); `balance_tail` (no K split) applies
+// split_count for the same sizes); `chained`: launched with programmatic
+// dependent launch after this library's previous kernel (launch_k);
+// `balance_tail` (no K split) applies
 // tail_plan, or for pairs with `tail_part` scratch of `tail_bytes` the
 // K-split tail when that leaves the shorter last round (a tail unit costs
 // 1/splits of a tile plus about a tenth of one for its partial tile and the
@@ -367,7 +403,7 @@ bool cluster_fits(int dev, int sms, int s, int count) {
 // (clusters of two).
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4, bool PAIR = false>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
-                     sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool balance_tail = false,
+                     sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool chained, bool balance_tail = false,
                      float* tail_part = nullptr, size_t tail_bytes = 0, const char* tail_name = nullptr) {
   using namespace sambay::tc;
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
@@ -472,38 +508,13 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   const int units = std::min(g.tiles, slots);
   {
     ProfScope ps(name, st);
-    if (PAIR) {
-      cudaLaunchConfig_t lc = {};
-      lc.gridDim = dim3(2 * units);
-      lc.blockDim = dim3(gemm_threads(EW));
-      lc.dynamicSmemBytes = C::kSmem;
-      lc.stream = st;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = 2;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      lc.attrs = at;
-      lc.numAttrs = 1;
-      if (cudaLaunchKernelEx(&lc, kern, ta, tb, tb2, taux, tout, g) != cudaSuccess) return SAMBAY_ERR_CUDA;
-    } else if (g.csplit) {
-      // one unit per CTA; the splits of a tile are one cluster
-      cudaLaunchConfig_t lc = {};
-      lc.gridDim = dim3(g.tiles);
-      lc.blockDim = dim3(gemm_threads(EW));
-      lc.dynamicSmemBytes = C::kSmem;
-      lc.stream = st;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = g.splits;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      lc.attrs = at;
-      lc.numAttrs = 1;
-      if (cudaLaunchKernelEx(&lc, kern, ta, tb, tb2, taux, tout, g) != cudaSuccess) return SAMBAY_ERR_CUDA;
-    } else {
-      kern<<<units, gemm_threads(EW), C::kSmem, st>>>(ta, tb, tb2, taux, tout, g);
-    }
+    // PAIR: one unit per cluster of two; cluster split-K: one cluster of
+    // `splits` CTAs per tile; otherwise one unit per CTA
+    const int grid = PAIR ? 2 * units : g.csplit ? g.tiles : units;
+    const int cluster = PAIR ? 2 : g.csplit ? g.splits : 1;
+    if (launch_k(kern, dim3(grid), dim3(gemm_threads(EW)), C::kSmem, st, chained, cluster, ta, tb, tb2, taux,
+                 tout, g) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
   }
   if constexpr (PAIR) if (ktail > 0) {
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
@@ -511,7 +522,8 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
     auto rk = tail_reduce_kernel<BN, C::kBMT, KIND>;
     SAMBAY_MAX_CARVEOUT(rk, dev);
     ProfScope ps(tail_name ? tail_name : "gemm_tail_reduce", st);
-    rk<<<grid_for(work, 256, sms), 256, 0, st>>>(g, ktail);
+    if (launch_k(rk, dim3(grid_for(work, 256, sms)), dim3(256), 0, st, true, 1, g, ktail) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
@@ -582,10 +594,10 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     gx.b_k_wrap = Di;
     const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
     constexpr int P = sambay::tc::EPI_F32_PARTIAL;
-    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
-    else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st)));
+    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+    else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
     {
       auto k8 = sambay::scan::xdbl_reduce_kernel<8>;
       auto k1 = sambay::scan::xdbl_reduce_kernel<1>;
@@ -593,10 +605,10 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
       SAMBAY_MAX_CARVEOUT(k1, dev);
       const int Lseq = static_cast<int>(rows / d->batch), nrows = static_cast<int>(rows);
       ProfScope ps_reduce("xdbl_reduce", st);
-      if (L.splits >= 16)
-        k8<<<grid_for(stride / 4 * 8, 256, sms), 256, 0, st>>>(part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx);
-      else
-        k1<<<grid_for(stride / 4, 256, sms), 256, 0, st>>>(part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx);
+      const bool many = L.splits >= 16;
+      if (launch_k(many ? k8 : k1, dim3(grid_for(stride / 4 * (many ? 8 : 1), 256, sms)), dim3(256), 0, st, true, 1,
+                   part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx) != cudaSuccess)
+        return SAMBAY_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
@@ -605,9 +617,9 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     gd.b_k_wrap = Rp;
     const Operand a_d{delta, rows, 2LL * Rp}, b_wdt{w->dt_proj_w, Di, R};
     if (rows <= sambay::tc::BM)   // one row tile (decode): narrower tiles, more CTAs
-      SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st)));
+      SAMBAY_TRY((run_tc<64, false, false, sambay::tc::EPI_SOFTPLUS, false>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st, true)));
     else
-      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st, true)));
+      SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st, true, true)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
     SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
@@ -665,8 +677,8 @@ sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cuda
   const ScanLayout ly(p.chp, sizeof(T));
   dim3 grid(p.nblk, p.B);
   ProfScope ps("selective_scan", st);
-  kern<<<grid, 8 * p.chp, ly.bytes, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+  return launch_k(kern, grid, dim3(8 * p.chp), ly.bytes, st, true, 1, p) == cudaSuccess ? SAMBAY_OK
+                                                                        : SAMBAY_ERR_CUDA;
 }
 
 template <typename T>
@@ -739,11 +751,13 @@ sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, con
   if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st));
   ProfScope ps("step_scan", st);
-  ss<<<grid_for(B * d->d_inner * 4, 256, 1 << 20), 256, 0, st>>>(
-      uc, reinterpret_cast<const float*>(ws + L.dt), reinterpret_cast<const float*>(ws + L.xdbl),
-      w->A, w->D, ssm_state, static_cast<T*>(m_t), d->batch, d->d_inner, d->dt_rank,
-      d->dt_rank + 2 * d->d_state);
-  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+  const cudaError_t e = launch_k(ss, dim3(grid_for(B * d->d_inner * 4, 256, 1 << 20)), dim3(256), 0, st, true, 1,
+                                 static_cast<const T*>(uc), reinterpret_cast<const float*>(ws + L.dt),
+                                 reinterpret_cast<const float*>(ws + L.xdbl), static_cast<const float*>(w->A),
+                                 static_cast<const float*>(w->D), ssm_state, static_cast<T*>(m_t),
+                                 static_cast<int>(d->batch), static_cast<int>(d->d_inner),
+                                 static_cast<int>(d->dt_rank), static_cast<int>(d->dt_rank + 2 * d->d_state));
+  return e == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ GMU
@@ -884,12 +898,12 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8, true>(
-      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, true,
-      tail, L.tail_bytes, "gmu_gate_tail")));
+      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, false,
+      true, tail, L.tail_bytes, "gmu_gate_tail")));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
   SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8, true>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
-      st, true, tail, L.tail_bytes, "gmu_out_tail")));
+      st, true, true, tail, L.tail_bytes, "gmu_out_tail")));
   return SAMBAY_OK;
 }
 
@@ -916,8 +930,8 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   g1.csplit = g2.csplit = 1;
   const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
 #define SAMBAY_STEP_GEMMS(BNV)                                                                   \
-  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, kStepMaxSplits, st))); \
-  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, kStepMaxSplits, st)));
+  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, kStepMaxSplits, st, false))); \
+  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, kStepMaxSplits, st, true)));
   if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
   else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
   else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }

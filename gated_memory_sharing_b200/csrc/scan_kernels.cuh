@@ -118,6 +118,8 @@ __device__ __forceinline__ void load4(const T* p, float (&x)[4]) {
 
 template <typename T, int CB>
 __global__ void __launch_bounds__(CB / 4 * (kConvTT / 4), 4) conv_silu_kernel(const ConvParams<T> p) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int ROWS = kConvTT + kK - 1;
   constexpr int EP = 16 / sizeof(T);          // elements per 16-byte piece
   constexpr int PPR = CB / EP;                // pieces per row
@@ -195,6 +197,8 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
                                    long long split_stride, float* __restrict__ xdbl,
                                    bf16* __restrict__ delta2, float* __restrict__ bcp, int L,
                                    int rows, int R, int Rp, int ldx) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long total4 = static_cast<long long>(rows) * ldx / 4;
   const int lane = threadIdx.x & 31, sub = lane % LPG;
   const long long warps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
@@ -276,6 +280,8 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
 // float32 path whose x_proj writes xdbl directly.  Thread: one (row, column).
 __global__ void bc_pairs_kernel(const float* __restrict__ xdbl, float* __restrict__ bcp, int L, int rows,
                                 int R, int ldx) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   if (i >= static_cast<long long>(rows) * 2 * kN) return;
   const int row = static_cast<int>(i / (2 * kN)), cc = static_cast<int>(i % (2 * kN));
@@ -484,6 +490,8 @@ __device__ __forceinline__ void scan_write_piece(const ScanParams<T>& p, const T
 
 template <typename T>
 __global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(const ScanParams<T> p) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t scan_smem_raw[];
   uint8_t* smem = scan_smem_raw;
   const ScanLayout ly(p.chp, sizeof(T));
@@ -608,6 +616,8 @@ __global__ void __launch_bounds__(256) step_conv_kernel(const T* __restrict__ u_
                                                         const T* __restrict__ conv_w,
                                                         const T* __restrict__ conv_b,
                                                         T* __restrict__ uc, int B, int Di) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int VEC = 16 / sizeof(T);
   constexpr int WV = VEC * kK * sizeof(T) / 16;   // 16-byte vectors per VEC windows
   const int groups = Di / VEC;
@@ -658,6 +668,8 @@ __global__ void __launch_bounds__(256) step_scan_kernel(const T* __restrict__ uc
                                                         const float* __restrict__ D,
                                                         float* __restrict__ h, T* __restrict__ m_t,
                                                         int B, int Di, int R, int ldx) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   const long long pair = idx >> 2;      // (b, c)
   const int q = static_cast<int>(idx & 3);

@@ -28,6 +28,8 @@ struct Args {
 
 template <int KIND>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const Args g) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float sa[16][64 + 4];
   __shared__ float sb[16][64 + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;

@@ -617,6 +617,10 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above touched only this CTA's shared memory and TMEM; global
+  // reads and writes wait for the kernel before this one on the stream
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -1004,6 +1008,8 @@ constexpr int kTailLanes = 4;
 
 template <int BN, int BMT, int KIND>
 __global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmArgs g, int ntail) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int Q = BN / 4, LPG = kTailLanes, PER = kMaxTailSplits / LPG;
   const int lane = threadIdx.x & 31, sub = lane % LPG;
   const long long total = static_cast<long long>(ntail) * BMT * Q;   // output float4s
