@@ -972,17 +972,38 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     const int R = (BM + g.splits - 1) / g.splits;
     const int r0 = c.split * R, r1 = min(BM, r0 + R);
     const int nrows = max(0, r1 - r0), ncols = min(c.bn, g.N - c.n0);
-    for (int e = threadIdx.x; e < nrows * ncols; e += blockDim.x) {
-      const int m = c.m * BM + r0 + e % nrows;   // consecutive threads: consecutive rows
-      const int n = c.n0 + e / nrows;
-      if (m >= g.M) continue;
-      const long long o = TRANS ? static_cast<long long>(n) * g.ldo + m : static_cast<long long>(m) * g.ldo + n;
-      float v = 0.0f;
-      for (int sp = 0; sp < g.splits; ++sp) v += __ldcg(g.partials + static_cast<long long>(sp) * g.split_stride + o);
-      float a = 0.0f;
-      if (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr))
-        a = to_f32(reinterpret_cast<const bf16*>(g.aux)[o]);
-      epi_store_one<KIND>(g, o, n, v, a);
+    const int total = nrows * ncols;
+    const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
+    // kRed elements per thread and pass, every load of a pass issued before
+    // its stores (a store may alias a later load as far as the compiler
+    // knows, which would otherwise chain one L2 round trip per element)
+    constexpr int kRed = 8;
+    for (int e0 = threadIdx.x; e0 < total; e0 += kRed * blockDim.x) {
+      long long o[kRed];
+      int nn[kRed];
+      bool live[kRed];
+      float v[kRed], a[kRed];
+#pragma unroll
+      for (int u = 0; u < kRed; ++u) {
+        const int e = e0 + u * static_cast<int>(blockDim.x);
+        const int m = c.m * BM + r0 + (e < total ? e % nrows : 0);   // consecutive threads: consecutive rows
+        nn[u] = c.n0 + (e < total ? e / nrows : 0);
+        live[u] = e < total && m < g.M;
+        o[u] = TRANS ? static_cast<long long>(nn[u]) * g.ldo + m : static_cast<long long>(m) * g.ldo + nn[u];
+        a[u] = has_aux && live[u] ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o[u]]) : 0.0f;
+        v[u] = 0.0f;
+      }
+      for (int sp = 0; sp < g.splits; ++sp) {
+        const float* part = g.partials + static_cast<long long>(sp) * g.split_stride;
+        float x[kRed];
+#pragma unroll
+        for (int u = 0; u < kRed; ++u) x[u] = live[u] ? __ldcg(part + o[u]) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < kRed; ++u) v[u] += x[u];
+      }
+#pragma unroll
+      for (int u = 0; u < kRed; ++u)
+        if (live[u]) epi_store_one<KIND>(g, o[u], nn[u], v[u], a[u]);
     }
   }
   if (warp == 1) {
