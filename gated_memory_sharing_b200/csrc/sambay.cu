@@ -186,7 +186,7 @@ ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
 }
 
 struct GmuWs {
-  size_t h, part, tail, tail_bytes, total;
+  size_t h, tail, tail_bytes, total;
 };
 
 constexpr int kStepMaxRows = 256;
@@ -200,12 +200,6 @@ GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
   size_t off = 0;
   w.h = off;
   off += round256(static_cast<size_t>(rows) * d->d_inner * io_bytes(d->io));
-  if (step && d->io == SAMBAY_BF16) {
-    // swap-AB split-K partials, room for kStepMaxSplits splits of either GEMM
-    // (output tiles over d_inner for GEMM1, d_model for GEMM2)
-    w.part = off;
-    off += round256(static_cast<size_t>(rows) * kStepMaxSplits * std::max(d->d_inner, d->d_model) * 4);
-  }
   if (!step && d->io == SAMBAY_BF16 && rows > 256) {
     // more than one 256-row tile: room for the K-split tail of either GEMM
     w.tail = off;
@@ -921,12 +915,12 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, residual, Y, w8, L, st);
   const int Dm = d->d_model, Di = d->d_inner, Bn = static_cast<int>(rows);
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
-  float* part = reinterpret_cast<float*>(w8 + L.part);
   // swap-AB: H^T = SiLU(W1 X^T) ⊙ M^T; W1 rows stream once through the tensor
-  // cores.  Split-K over clusters of CTAs (csplit): the splits of a tile meet
-  // at a cluster barrier and each finishes a slice of its rows.
-  auto g1 = tc_args(Di, Bn, Dm, H, Di, M, nullptr, part, rows * static_cast<long long>(Di));
-  auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual, nullptr, part, rows * static_cast<long long>(Dm));
+  // cores.  Split-K over clusters of CTAs (csplit): each split keeps its
+  // partial tile in shared memory; after a cluster barrier each CTA sums a
+  // slice of the tile's rows over the cluster (distributed shared memory).
+  auto g1 = tc_args(Di, Bn, Dm, H, Di, M);
+  auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual);
   g1.csplit = g2.csplit = 1;
   const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
 #define SAMBAY_STEP_GEMMS(BNV)                                                                   \

@@ -113,6 +113,21 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The shared::cluster address of this CTA's shared variable at `addr` in the
+// cluster's CTA `rank`, and a 16-byte load through it (distributed shared memory).
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 // TMA load into this CTA's shared memory whose bytes complete on the
 // leader CTA's barrier
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
@@ -481,6 +496,10 @@ struct Cfg {
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t kIdesc = idesc_bf16(kBMT, BN, A_MN, B_MN);
   static constexpr size_t kSmem = static_cast<size_t>(kFixed) + static_cast<size_t>(kStages) * kStageBytes;
+  // cluster split-K partial tile in the pipeline stages: BM rows of BN floats
+  // at a pitch of BN + 4 (16-byte rows whose starts step by 4 banks)
+  static constexpr int kCsplitPitch = BN + 4;
+  static constexpr bool kCsplitFits = BM * kCsplitPitch * 4 <= kStages * kStageBytes;
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
   static_assert(EW == 4 || EW == 8, "one or two epilogue warps per TMEM lane quarter");
@@ -549,6 +568,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs g) {
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   constexpr int S = C::kStages;
+  static_assert(!TRANS || C::kCsplitFits, "cluster split-K partial tile exceeds the pipeline stages");
   // work units: one per CTA, or one per CTA pair (cluster of 2)
   const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
   const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
@@ -881,6 +901,14 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             __stcg(reinterpret_cast<float4*>(part + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+        } else if (split && g.csplit) {
+          // cluster split-K: this split's partial tile stays in this CTA's
+          // (now idle) pipeline shared memory, row-major at kCsplitPitch; the
+          // cluster's CTAs read it there after the cluster barrier
+          float* dst = reinterpret_cast<float*>(smem) + (quarter * 32 + lane) * C::kCsplitPitch + ch * 32;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         } else if (split) {
           // this split's partial tile, summed in split order by the last CTA
           float* part = g.partials + static_cast<long long>(c.split) * g.split_stride;
@@ -963,48 +991,70 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
   else __syncthreads();
   tc_fence_after();
   if (!PAIR && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {
-    // cluster split-K: every CTA of the cluster has written its partial tile;
-    // CTA `split` now sums rows [split * R, +R) of the tile over the splits in
-    // split order and applies the final op
-    __threadfence();
+    // cluster split-K: every CTA of the cluster holds its partial tile in its
+    // shared memory; CTA `split` (cluster rank `split`) sums rows
+    // [split * R, +R) of the tile over the splits in split order, reading the
+    // peers' tiles 16 bytes at a time through distributed shared memory, and
+    // applies the final op.  Thread: 4 consecutive columns of one row,
+    // consecutive threads on consecutive rows.
     cluster_sync();
     const TileCoord c = tile_coord<BN>(g, blockIdx.x);
     const int R = (BM + g.splits - 1) / g.splits;
     const int r0 = c.split * R, r1 = min(BM, r0 + R);
     const int nrows = max(0, r1 - r0), ncols = min(c.bn, g.N - c.n0);
-    const int total = nrows * ncols;
+    const int total = nrows * ((ncols + 3) / 4);
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
-    // kRed elements per thread and pass, every load of a pass issued before
-    // its stores (a store may alias a later load as far as the compiler
-    // knows, which would otherwise chain one L2 round trip per element)
-    constexpr int kRed = 8;
+    const uint32_t base = smem_u32(smem);
+    // kRed elements per thread and pass, every load of a pass issued first
+    constexpr int kRed = 4;
     for (int e0 = threadIdx.x; e0 < total; e0 += kRed * blockDim.x) {
-      long long o[kRed];
-      int nn[kRed];
+      int mm[kRed], nn[kRed];
+      uint32_t off[kRed];
       bool live[kRed];
-      float v[kRed], a[kRed];
+      float4 v[kRed];
+      float a[kRed][4];
 #pragma unroll
       for (int u = 0; u < kRed; ++u) {
         const int e = e0 + u * static_cast<int>(blockDim.x);
-        const int m = c.m * BM + r0 + (e < total ? e % nrows : 0);   // consecutive threads: consecutive rows
-        nn[u] = c.n0 + (e < total ? e / nrows : 0);
-        live[u] = e < total && m < g.M;
-        o[u] = TRANS ? static_cast<long long>(nn[u]) * g.ldo + m : static_cast<long long>(m) * g.ldo + nn[u];
-        a[u] = has_aux && live[u] ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o[u]]) : 0.0f;
-        v[u] = 0.0f;
+        const int lr = r0 + (e < total ? e % nrows : 0);
+        const int lc = 4 * (e < total ? e / nrows : 0);
+        mm[u] = c.m * BM + lr;
+        nn[u] = c.n0 + lc;
+        live[u] = e < total && mm[u] < g.M;
+        off[u] = static_cast<uint32_t>(lr * C::kCsplitPitch + lc) * 4u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const long long o = TRANS ? static_cast<long long>(nn[u] + k) * g.ldo + mm[u]
+                                    : static_cast<long long>(mm[u]) * g.ldo + nn[u] + k;
+          a[u][k] = has_aux && live[u] && nn[u] + k < g.N ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o]) : 0.0f;
+        }
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       for (int sp = 0; sp < g.splits; ++sp) {
-        const float* part = g.partials + static_cast<long long>(sp) * g.split_stride;
-        float x[kRed];
+        const uint32_t peer = mapa_shared(base, static_cast<uint32_t>(sp));
+        float4 x[kRed];
 #pragma unroll
-        for (int u = 0; u < kRed; ++u) x[u] = live[u] ? __ldcg(part + o[u]) : 0.0f;
+        for (int u = 0; u < kRed; ++u) x[u] = ld_dsmem_f32x4(peer + off[u]);
 #pragma unroll
-        for (int u = 0; u < kRed; ++u) v[u] += x[u];
+        for (int u = 0; u < kRed; ++u) {
+          v[u].x += x[u].x; v[u].y += x[u].y; v[u].z += x[u].z; v[u].w += x[u].w;
+        }
       }
 #pragma unroll
-      for (int u = 0; u < kRed; ++u)
-        if (live[u]) epi_store_one<KIND>(g, o[u], nn[u], v[u], a[u]);
+      for (int u = 0; u < kRed; ++u) {
+        if (!live[u]) continue;
+        const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (nn[u] + k >= g.N) break;
+          const long long o = TRANS ? static_cast<long long>(nn[u] + k) * g.ldo + mm[u]
+                                    : static_cast<long long>(mm[u]) * g.ldo + nn[u] + k;
+          epi_store_one<KIND>(g, o, nn[u] + k, w[k], a[u][k]);
+        }
+      }
     }
+    // no CTA leaves (and frees its shared memory) while a peer still reads it
+    cluster_sync();
   }
   if (warp == 1) {
     if (PAIR)

@@ -74,7 +74,8 @@ def test_workspace_queries(lib):
     # CTA pair of 148 SMs for a GEMM's K-split tail
     assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2) + r256(74 * 256 * 256 * 4)
     assert abi.gmu_forward_workspace(d, 256) == r256(256 * 5120 * 2)
-    assert abi.gmu_step_workspace(d, 64) > 64 * 5120 * 2
+    # H only: the decode GEMMs reduce their K splits in shared memory
+    assert abi.gmu_step_workspace(d, 64) == r256(64 * 5120 * 2)
     # invalid or unsupported dims -> 0
     assert abi.sambay_scan_prefill_workspace(abi.make_dims(1, 16, 64, 128, 8, 4, 8, abi.BF16)) == 0
     assert abi.sambay_scan_prefill_workspace(abi.make_dims(0, 16, 64, 128)) == 0
