@@ -39,13 +39,14 @@ WORKLOAD = "prefill_b1_l2048"
 # changed since its capture has no entry (reported as null).
 DRAM_TRAFFIC = {
     # profiles/prefill_b1_l2048_launches.md (bench.py --steps 3 --warmup 3 --no-cpu-baseline --no-decode)
-    "conv_silu": 21034240 + 86016,
-    "x_proj": 43944448 + 768,
+    "conv_silu": 21034496 + 98560,
+    "x_proj": 43948032 + 768,
     "xdbl_reduce": 14177280 + 0,
-    "dt_proj": 3315712 + 0,
-    "selective_scan": 84559872 + 2316288,
-    "gmu_gate_gemm": 57750784 + 175872,
-    "gmu_out_gemm": 47247360 + 77824,
+    "dt_proj": 3319296 + 0,
+    "selective_scan": 84559616 + 2436352,
+    "gmu_gate_gemm": 57772544 + 907008,
+    "gmu_out_gemm": 47287040 + 243456,
+    "gmu_out_tail": 18881792 + 0,
 }
 METRIC = "scan+GMU prefill tokens/s"
 UNIT = "tokens/s"
