@@ -29,6 +29,10 @@
  *     (no TF32); SAMBAY_BF16 runs the tcgen05 tensor-core kernels.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and never synchronise, except sambay_device_status.
+ *     A call's first kernel orders after everything queued before it on the
+ *     stream; its later kernels use programmatic dependent launch, starting
+ *     while the previous kernel of the same call finishes and waiting for it
+ *     before they touch memory.
  *   - Argument errors (NULL pointers, bad or unsupported sizes, misaligned
  *     pointers, short workspace) are detected on the host BEFORE any launch,
  *     and return a status without touching the device.  Launch failures
@@ -154,7 +158,10 @@ SAMBAY_API sambay_status sambay_scan_step(const sambay_scan_weights* w, const sa
  *   residual [rows, Dm] io or NULL;  Y [rows, Dm] io out (may alias
  *   residual, must not alias X unless X == residual, nor M).
  * Two tensor-core GEMMs: G = X W1^T with SiLU(G) ⊙ M fused into its
- * epilogue (H, io, kept in ws), then H W2 with the residual fused.
+ * epilogue (H, io, kept in ws), then H W2 with the residual fused.  In bf16
+ * with more than 256 rows, ws also holds the fp32 partial tiles of a GEMM
+ * whose last round of tiles is split along K (summed in a fixed order, so
+ * results do not vary from run to run).
  */
 SAMBAY_API sambay_status gmu_forward(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
                           const void* W1, const void* W2, const void* residual, void* Y,
@@ -164,7 +171,9 @@ SAMBAY_API sambay_status gmu_forward(const sambay_dims* dims, int64_t rows, cons
  * gmu_step - the GMU for one decode token of `rows` sequences (rows <= 256)
  * [GMU], [FRAME] (O(d_h) memory per token: the weights are streamed once).
  * Same arguments and semantics as gmu_forward; a weight-streaming kernel
- * pair (swap-AB tensor-core GEMV with split-K) instead of the tiled GEMMs.
+ * pair (swap-AB tensor-core GEMV with split-K over a cluster of CTAs, the
+ * splits summed in a fixed order through distributed shared memory) instead
+ * of the tiled GEMMs; ws holds only H.
  */
 SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
                        const void* W1, const void* W2, const void* residual, void* Y,
