@@ -42,4 +42,9 @@ from .sambay_ref import (  # noqa: F401
     gmu_layers_ref,
     mixing_matrix_ref,
     lifted_gmu_ref,
+    round_bf16,
+    mamba_layer_ref,
+    mlp_representation_ref,
+    sambay_mlp_gmu_ref,
+    cross_attention_decode_ref,
 )

@@ -33,6 +33,11 @@ __all__ = [
     "gmu_layers_ref",
     "mixing_matrix_ref",
     "lifted_gmu_ref",
+    "round_bf16",
+    "mamba_layer_ref",
+    "mlp_representation_ref",
+    "sambay_mlp_gmu_ref",
+    "cross_attention_decode_ref",
 ]
 
 
@@ -183,6 +188,25 @@ def scan_step_ref(u_t, w, ssm_state, conv_state):
 
 
 # --------------------------------------------------------------------------
+# The bf16 I/O type
+# --------------------------------------------------------------------------
+
+def round_bf16(x):
+    """Round to the nearest bfloat16 value, ties to even; float64 out.
+
+    bfloat16 keeps 8 significant bits: for |x| in [2^(e-1), 2^e) the spacing
+    is 2^(e-8), and below the smallest normal 2^-126 it stays 2^-133.  Only
+    used where a caller-visible tensor of a bf16 workload passes between two
+    calls (the I/O of the cross-decoder's layers); finite inputs only.
+    """
+    x = _f64(x)
+    _, e = np.frexp(x)                      # x = m 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                 # normal range of bf16: 2^-126 and up
+    ulp = np.ldexp(1.0, e - 8)
+    return np.rint(x / ulp) * ulp           # np.rint rounds half to even
+
+
+# --------------------------------------------------------------------------
 # Gated Memory Unit (Paper-Notes, 方法详解 > 关键设计)
 # --------------------------------------------------------------------------
 
@@ -202,16 +226,25 @@ def gmu_ref(X, M, W1, W2, residual=False):
     return Y, G, H
 
 
-def gmu_layers_ref(X, M, W1s, W2s):
+def gmu_layers_ref(X, M, W1s, W2s, io_round=False):
     """Cross-decoder sharing: one memory readout M feeds a stack of GMUs.
 
     X_{l+1} = X_l + GMU_l(X_l, M) for each (W1_l, W2_l); every layer reads the
     same M (Paper-Notes, 整体框架: the cross-decoder's GMU layers reuse the
     last SSM layer's token-mixing output).  Returns the final X.
+
+    ``io_round``: the layers exchange X (and read M) as bfloat16 tensors, the
+    I/O type of the bf16 workloads, so each layer's input is the bf16 rounding
+    of the previous layer's exact output (:func:`round_bf16`); the arithmetic
+    inside a layer stays exact.  Without it, X is carried exactly from layer
+    to layer.
     """
     X = _f64(X)
+    M = round_bf16(M) if io_round else _f64(M)
     for W1, W2 in zip(W1s, W2s):
         X, _, _ = gmu_ref(X, M, W1, W2, residual=True)
+        if io_round:
+            X = round_bf16(X)
     return X
 
 
@@ -261,3 +294,82 @@ def lifted_gmu_ref(uc, G, mix, W2):
     At = np.einsum("ik,kij->ijk", G, mix)          # [L, L, Di]
     H = np.einsum("ijk,jk->ik", At, uc)            # [L, Di]
     return H @ W2
+
+
+# --------------------------------------------------------------------------
+# Around the path: the Mamba layer that produces M, and the two neighbours of
+# the GMU in the cross-decoder
+# --------------------------------------------------------------------------
+
+def mamba_layer_ref(X, w, W_in, W_z, W_out, ssm_state=None, conv_state=None, residual=True):
+    """The whole Mamba layer whose scan readout is the shared memory M.
+
+    Mamba block (Gu & Dao 2023, section 3.4): the input is projected into two
+    branches, x = X W_in^T (the scan input u) and z = X W_z^T (the gate); the
+    scan of u gives y, the layer output is (y ⊙ SiLU(z)) W_out.  The Samba
+    self-decoder stacks such layers (Paper-Notes, 方法详解 > 整体框架), and M is
+    the last one's y before its own gate (reading: the GMU's gate takes the
+    place of SiLU(z), so M is the pre-gate readout).
+
+    X [B, L, Dm]; W_in, W_z [Di, Dm] (the x and z halves of in_proj, used
+    transposed); W_out [Di, Dm], multiplying on the right (out_proj's weight
+    transposed).  Returns dict(out [B, L, Dm] (+X when ``residual``), M = y,
+    z, u, ssm_state, conv_state).
+    """
+    X = _f64(X)
+    u = X @ _f64(W_in).T
+    z = X @ _f64(W_z).T
+    r = scan_prefill_ref(u, w, ssm_state, conv_state)
+    out = (r["M"] * silu(z)) @ _f64(W_out)
+    if residual:
+        out = out + X
+    return dict(out=out, M=r["M"], z=z, u=u, ssm_state=r["ssm_state"], conv_state=r["conv_state"])
+
+
+def mlp_representation_ref(X, W_g, W_u):
+    """The intermediate representation of a SwiGLU MLP: SiLU(X W_g^T) ⊙ (X W_u^T).
+
+    SambaY-MLP (Paper-Notes, 实验关键数据 > 消融实验, row "SambaY-MLP") lets the
+    GMUs gate an MLP representation instead of the SSM readout; reading: the
+    hidden activation of the self-decoder's last MLP, whose SwiGLU form is the
+    Samba MLP.  X [T, Dm]; W_g, W_u [Dff, Dm].  Returns [T, Dff].
+    """
+    X = _f64(X)
+    return silu(X @ _f64(W_g).T) * (X @ _f64(W_u).T)
+
+
+def sambay_mlp_gmu_ref(X_cross, X_self, W_g, W_u, W1, W2, residual=False):
+    """A SambaY-MLP GMU layer: the memory is the MLP representation of the
+    self-decoder's input X_self, gated by the cross-decoder's X_cross.
+    Returns (Y, M)."""
+    M = mlp_representation_ref(X_self, W_g, W_u)
+    Y, _, _ = gmu_ref(X_cross, M, W1, W2, residual=residual)
+    return Y, M
+
+
+def cross_attention_decode_ref(q, K, V, scale=None):
+    """One decode query per sequence attending over the single KV cache.
+
+    The cross-decoder layers that the GMU does not replace attend to the KV
+    cache the self-decoder's full-attention layer wrote once (Paper-Notes,
+    方法详解 > 整体框架; 研究背景与动机: the O(d_kv N) memory I/O per decoded
+    token that the GMU avoids).  Standard softmax attention with grouped
+    query heads:
+
+        out[b, h] = sum_j softmax_j(scale q[b, h] . K[b, j, h // G]) V[b, j, h // G]
+
+    q [B, Hq, dh]; K, V [B, N, Hkv, dh] with G = Hq / Hkv; scale defaults to
+    1 / sqrt(dh).  Returns [B, Hq, dh].
+    """
+    q, K, V = map(_f64, (q, K, V))
+    Bsz, Hq, dh = q.shape
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    s = (1.0 / np.sqrt(dh)) if scale is None else float(scale)
+    Kq = np.repeat(K, G, axis=2)                       # [B, N, Hq, dh]
+    Vq = np.repeat(V, G, axis=2)
+    logits = np.einsum("bhd,bnhd->bhn", q, Kq) * s      # [B, Hq, N]
+    logits = logits - logits.max(axis=-1, keepdims=True)
+    p = np.exp(logits)
+    p = p / p.sum(axis=-1, keepdims=True)
+    return np.einsum("bhn,bnhd->bhd", p, Vq)
