@@ -1,14 +1,23 @@
 """Benchmark of the SambaY scan + Gated Memory Unit hot path on B200.
 
-One step = one pass of the prefill hot path over one batch: the Mamba
-selective scan of a 2048-token prompt (batch 1, d_inner 5120, d_state 16,
-conv 4, dt_rank 160) writing the memory readout M, then one GMU layer
-Y = (M ⊙ SiLU(X W1^T)) W2 with d_model 2560, in bfloat16 I/O with float32
-accumulation and state.  Metric: tokens/s over the step.  A decode
-sub-benchmark (64 sequences, one token each per step: scan step + GMU step)
-is reported beside it.
+The headline step is one pass of the prefill hot path over one batch: the
+Mamba selective scan of a 2048-token prompt (batch 1, d_model 2560, d_inner
+5120, d_state 16, conv 4, dt_rank 160) writing the memory readout M, then one
+GMU layer Y = (M ⊙ SiLU(X W1^T)) W2, in bfloat16 I/O with float32
+accumulation and state.  Metric: tokens/s.  The other seeded workloads of the
+method are measured in the same run and reported under "workloads":
+
+  decode_b64               64 sequences, 2048-token prompt, then decode steps
+                           (scan step + one GMU layer with residual); the full
+                           32768-step horizon is also timed back to back
+  long_prefill_b4_l32768   4 x 32768 tokens: scan + one GMU layer
+  sharing_b2_l8192         one scan of 2 x 8192 tokens whose M feeds 8 GMU
+                           layers (X <- X + GMU_l(X, M))
+  sharing_decode_b16       16 sequences decoding through the scan step and
+                           the 8 GMU layers
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--only-headline] [--no-cpu-baseline]
 
 N > 1 runs under torchrun, one process per GPU, each an independent replica
 (weak scaling: the sequences of different ranks share nothing, so there is
@@ -33,29 +42,31 @@ sys.path.insert(0, ROOT)
 
 from gated_memory_sharing_b200 import synth  # noqa: E402
 
-WORKLOAD = "prefill_b1_l2048"
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
-# kernel, from one ncu capture of the benchmarked workload (profiles/); a kernel
-# changed since its capture has no entry (reported as null).
-DRAM_TRAFFIC = {
-    # profiles/prefill_b1_l2048_launches.md (bench.py --steps 3 --warmup 3 --no-cpu-baseline --no-decode)
-    "conv_silu": 21034496 + 98560,
-    "x_proj": 43948032 + 768,
-    "xdbl_reduce": 14177280 + 0,
-    "dt_proj": 3319296 + 0,
+HEADLINE = "prefill_b1_l2048"
+WORKLOADS = ("prefill_b1_l2048", "decode_b64", "long_prefill_b4_l32768", "sharing_b2_l8192",
+             "sharing_decode_b16")
+UNIT = "tokens/s"
+METRICS = {
+    "prefill_b1_l2048": "scan+GMU prefill tokens/s",
+    "decode_b64": "scan+GMU decode tokens/s",
+    "long_prefill_b4_l32768": "scan+GMU prefill tokens/s",
+    "sharing_b2_l8192": "scan+8xGMU prefill tokens/s",
+    "sharing_decode_b16": "scan+8xGMU decode tokens/s",
+}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from an
+# earlier ncu capture of the headline workload, for kernels unchanged since
+# that capture; any other kernel reports null.
+DRAM_TRAFFIC_EARLIER_CAPTURE = {
     "selective_scan": 84559616 + 2436352,
     "gmu_gate_gemm": 57772544 + 907008,
-    "gmu_out_gemm": 47287040 + 243456,
-    "gmu_out_tail": 18881792 + 0,
 }
-METRIC = "scan+GMU prefill tokens/s"
-UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 # Special-function-unit exp2 rate per SM per clock (4 lanes per sub-partition
 # x 4 sub-partitions; checked on this B200 with an ex2.approx throughput probe)
 SFU_EX2_PER_SM_CLK = 16
 L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
+DECODE_RING = 256            # decode inputs cycle through this many steps
 
 
 class L2Flush:
@@ -72,8 +83,6 @@ class L2Flush:
     def __call__(self, i):
         self.w.fill_(float(i))
         self.sink = self.r.amax()
-DECODE_BATCH = 64
-DECODE_RING = 64             # decode steps per captured graph
 
 
 def load_peaks():
@@ -88,7 +97,7 @@ def load_peaks():
 # --------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples while the timed regions run."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -188,52 +197,128 @@ def barrier(world):
         dist.barrier()
 
 
-# --------------------------------------------------------------------- reference arm
+def dev_normal(shape, seed, device):
+    """Seeded N(0, 1) bf16 draws made on the device (the GPU arm's activations;
+    the weights come from the shared seeded generator module)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def workload_dims(name):
+    """(dims, seed, gmu layers, decode batch or None, decode prompt) of a bench workload."""
+    if name == "sharing_decode_b16":
+        d, seed = synth.workload("sharing_b2_l8192")
+        return (synth.Dims(synth.SHARING_DECODE_BATCH, 1024, d.d_model, d.d_inner, d.d_state, d.d_conv,
+                           d.dt_rank, synth.BF16), seed, synth.SHARING_LAYERS, True)
+    d, seed = synth.workload(name)
+    if name == "decode_b64":
+        return d, seed, 1, True
+    layers = synth.SHARING_LAYERS if name == "sharing_b2_l8192" else 1
+    return d, seed, layers, False
+
+
+def config_of(name, d, layers, decode):
+    c = {"workload": name, "batch": d.batch, "seq_len": d.seqlen, "d_model": d.d_model,
+         "d_inner": d.d_inner, "d_state": d.d_state, "d_conv": d.d_conv, "dt_rank": d.dt_rank,
+         "gmu_layers": layers}
+    if decode:
+        c["prompt"] = d.seqlen
+        c.pop("seq_len")
+        c["decode_steps"] = synth.DECODE_STEPS.get("decode_b64" if name == "decode_b64" else "sharing_b2_l8192")
+    return c
+
+
+# --------------------------------------------------------------------- the oracle on the host
+
+def _oracle_prefill(u, X, w, gws, residual):
+    from oracle import sambay_ref as ref
+    r = ref.scan_prefill_ref(u, w)
+    M = r["M"].reshape(-1, u.shape[-1])
+    if len(gws) == 1:
+        ref.gmu_ref(X, M, gws[0]["W1"], gws[0]["W2"], residual=residual)
+    else:
+        ref.gmu_layers_ref(X, M, [g["W1"] for g in gws], [g["W2"] for g in gws])
+
+
+def cpu_baseline(name, budget_s=8.0, reps_max=4):
+    """The oracle as it stands, timed on this host on a bounded sample of the
+    workload: whole prefill steps where affordable, otherwise a prefix of one
+    sequence; decode steps of every sequence of the batch."""
+    from oracle import sambay_ref as ref
+    d, seed, layers, decode = workload_dims(name)
+    w = synth.scan_weights(d, seed)
+    gws = [synth.gmu_weights(d, seed, layer=l) for l in range(layers)]
+    cores = len(os.sched_getaffinity(0))
+    if decode:
+        B = d.batch
+        dd = synth.Dims(B, 16, d.d_model, d.d_inner, d.d_state, d.d_conv, d.dt_rank, synth.BF16)
+        r = ref.scan_prefill_ref(synth.scan_inputs(dd, seed, tag="u_cpu"), w)
+        h, cs = r["ssm_state"], r["conv_state"]
+        steps, t0 = 0, time.perf_counter()
+        while steps < 64 and (steps == 0 or time.perf_counter() - t0 < budget_s):
+            u_t = synth.scan_inputs(dd, seed + steps, seqlen=1, tag="u_cpu_t")[:, 0]
+            x = synth.gmu_inputs(dd, seed + steps, rows=B, tag="x_cpu_t")
+            m, h, cs = ref.scan_step_ref(u_t, w, h, cs)
+            ref.gmu_layers_ref(x, m, [g["W1"] for g in gws], [g["W2"] for g in gws])
+            steps += 1
+        el = time.perf_counter() - t0
+        return {"value": steps * B / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"{steps} decode steps of all {B} sequences (scan step + {layers} GMU layer(s)) "
+                          f"after a 16-token prompt, {el:.1f} s of float64 NumPy"}
+    if d.tokens <= 4096:
+        u, X, tokens = synth.scan_inputs(d, seed), synth.gmu_inputs(d, seed), d.tokens
+        what = f"the whole step ({tokens} tokens)"
+    else:
+        L = 512
+        u = synth.scan_inputs(d, seed, batch=1, seqlen=L)
+        X = synth.gmu_inputs(d, seed, rows=L)
+        tokens = L
+        what = f"the first {L} tokens of one sequence"
+    reps, t0 = 0, time.perf_counter()
+    while reps < reps_max and (reps == 0 or time.perf_counter() - t0 < budget_s):
+        _oracle_prefill(u, X, w, gws, residual=layers > 1)
+        reps += 1
+    el = time.perf_counter() - t0
+    return {"value": reps * tokens / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{what}: scan + {layers} GMU layer(s), x {reps}, {el:.1f} s of float64 NumPy"}
+
 
 def run_reference(args, world, rank):
-    """The float64 oracle on the host cores, on a bounded sample per step."""
+    """--impl reference: the float64 oracle on the host cores, each step a
+    bounded sample of the headline workload (rank 0 only)."""
     if rank != 0:
         return
-    from oracle import sambay_ref as ref
-    d, seed = synth.workload(WORKLOAD)
-    w = synth.scan_weights(d, seed)
-    gw = synth.gmu_weights(d, seed)
-    sample = 256
-    u = synth.scan_inputs(d, seed, seqlen=sample)
-    X = synth.gmu_inputs(d, seed, rows=sample)
-
-    def step():
-        r = ref.scan_prefill_ref(u, w)
-        ref.gmu_ref(X, r["M"][0], gw["W1"], gw["W2"])
-
+    name = args.workload
+    d, seed, layers, decode = workload_dims(name)
     for _ in range(args.warmup):
-        step()
+        cpu_baseline(name, budget_s=0.0, reps_max=1)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
+    vals = [cpu_baseline(name, budget_s=0.0, reps_max=1) for _ in range(args.steps)]
     el = time.perf_counter() - t0
-    value = args.steps * sample / el
-    cores = len(os.sched_getaffinity(0))
-    desc = f"first {sample} tokens of the {d.seqlen}-token prompt (scan + GMU rows) per step"
+    value = statistics.mean(v["value"] for v in vals)
+    base = dict(vals[0])
+    base["value"] = value
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "impl": "reference", "metric": METRICS[name], "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": d.batch, "seq_len": d.seqlen,
-                   "d_model": d.d_model, "d_inner": d.d_inner, "d_state": d.d_state,
-                   "sample_tokens": sample},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "config": config_of(name, d, layers, decode),
+        "cpu_baseline": base,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
-def kernel_work(name, d, sms, peaks, peak_kind):
-    """(bound, algorithmic units per launch, unit, peak) of one kernel of the
-    prefill step on dims d.  Algorithmic = what the method must compute or move
-    once: exps for the scan, 2*M*N*K flops for the GEMMs, bytes read + written
-    by the memory-bound kernels (inputs once, outputs once)."""
+# --------------------------------------------------------------------- roofline bookkeeping
+
+def prefill_kernel_work(name, d, layers, sms, peaks, peak_kind):
+    """(bound, algorithmic units per launch, unit, peak, note) of one kernel of a
+    prefill step.  Algorithmic = what the method must compute or move once:
+    exps for the scan, 2*M*N*K flops for a GMU GEMM (the out GEMM's K-split
+    tail reduction counts as part of the out GEMM), bytes read + written by the
+    memory-bound kernels (inputs once, outputs once)."""
     T, Di, Dm, N, R = d.tokens, d.d_inner, d.d_model, d.d_state, d.dt_rank
     ldx, Rp = R + 2 * N, (R + 63) // 64 * 64
     hbm = peaks["hbm_gbs"]
@@ -241,7 +326,7 @@ def kernel_work(name, d, sms, peaks, peak_kind):
         peak = SFU_EX2_PER_SM_CLK * sms * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e9
         return "alu", T * Di * N, "Gexp/s", peak, \
             f"SFU ex2: {SFU_EX2_PER_SM_CLK}/SM/clk x {sms} SMs x max SM clock ({peak_kind} clock)"
-    if name in ("gmu_gate_gemm", "gmu_out_gemm"):
+    if name in ("gmu_gate_gemm", "gmu_gate_gemm+tail", "gmu_out_gemm", "gmu_out_gemm+tail"):
         return "tensor", 2.0 * T * Dm * Di, "TFLOP/s", peaks["bf16_tflops"], f"{peak_kind} burst bf16"
     if name == "conv_silu":      # u in (bf16), uc split pair out (2 x bf16)
         return "hbm", T * Di * (2 + 4), "GB/s", hbm, f"{peak_kind} HBM copy"
@@ -254,32 +339,298 @@ def kernel_work(name, d, sms, peaks, peak_kind):
     return None
 
 
-def cpu_baseline_oracle(min_seconds=10.0, max_reps=4):
-    """The oracle as it stands, on the full benchmark step, timed on this host."""
-    from oracle import sambay_ref as ref
-    d, seed = synth.workload(WORKLOAD)
+def merge_tails(per_kernel):
+    """A GEMM's K-split tail reduce finishes that GEMM: fold its time into the
+    GEMM's entry (reported as '<gemm>+tail')."""
+    out = dict(per_kernel)
+    for gemm, tail in (("gmu_out_gemm", "gmu_out_tail"), ("gmu_gate_gemm", "gmu_gate_tail")):
+        if gemm in out and tail in out:
+            a, b = out.pop(gemm), out.pop(tail)
+            n = min(len(a), len(b))
+            out[gemm + "+tail"] = [a[i] + b[i] for i in range(n)]
+    return out
+
+
+def decode_bytes(d, B, layers):
+    """Algorithmic bytes of one decode step: the fp32 state and the conv window
+    read and written, every weight read once, the activations in and out."""
+    Di, Dm, N, K, R = d.d_inner, d.d_model, d.d_state, d.d_conv, d.dt_rank
+    state = B * Di * N * 4 * 2 + B * Di * K * 2 * 2
+    scan_w = (R + 2 * N) * Di * 2 + Di * R * 2 + Di * (K + 1) * 2 + Di * N * 4 + 2 * Di * 4
+    gmu_w = layers * 2 * Di * Dm * 2
+    acts = B * (2 * Di + 2 * Dm) * 2
+    return state + scan_w + gmu_w + acts
+
+
+# --------------------------------------------------------------------- our arm: prefill
+
+def bench_prefill(args, ctx, name):
+    import torch
+    from gated_memory_sharing_b200 import abi
+    from gated_memory_sharing_b200.layers import GMULayer, ScanLayer
+    world, rank, device, flush, stream, peaks, peak_kind, sms = ctx
+    d, seed, layers, _ = workload_dims(name)
     w = synth.scan_weights(d, seed)
-    gw = synth.gmu_weights(d, seed)
-    u = synth.scan_inputs(d, seed)
-    X = synth.gmu_inputs(d, seed)
-    reps, t0 = 0, time.perf_counter()
-    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_seconds):
-        r = ref.scan_prefill_ref(u, w)
-        ref.gmu_ref(X, r["M"][0], gw["W1"], gw["W2"])
-        reps += 1
-    el = time.perf_counter() - t0
-    return {"value": reps * d.tokens / el, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
-            "kind": "oracle",
-            "sample": f"the whole step ({d.tokens} tokens: scan + one GMU layer) x {reps}, "
-                      f"{el:.1f} s of float64 NumPy"}
+    gws = [synth.gmu_weights(d, seed, layer=l) for l in range(layers)]
+    scan = ScanLayer(w, d.d_model, abi.BF16)
+    gmus = [GMULayer(g["W1"], g["W2"], abi.BF16) for g in gws]
+    # each rank: its own sequences (weak scaling), the same weights
+    u = dev_normal((d.batch, d.seqlen, d.d_inner), seed + 7919 * rank, device)
+    X0 = dev_normal((d.tokens, d.d_model), seed + 7919 * rank + 1, device)
+    T, Di = d.tokens, d.d_inner
+    M = torch.empty_like(u)
+    X = X0.clone()
+    Y = torch.empty_like(X0)
+    h, cs = scan.new_state(d.batch)
+    residual = layers > 1
+
+    def step():
+        scan.prefill(u, h, cs, M=M, fresh=True)
+        if residual:
+            for g in gmus:
+                g.forward(X, M.view(T, Di), residual=True, Y=X)
+        else:
+            gmus[0].forward(X, M.view(T, Di), residual=False, Y=Y)
+
+    def reset():
+        if residual:
+            X.copy_(X0)
+
+    for _ in range(max(args.warmup, 3)):
+        reset()
+        step()
+    torch.cuda.synchronize()
+    assert abi.sambay_device_status() == 0
+    steps = args.steps if name == HEADLINE else max(3, min(args.steps, 10))
+
+    # ---- device-resident timed region: K steps, L2 flushed between steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        reset()
+        flush(i)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    value = world * steps * T / (total_ms / 1e3)
+
+    # ---- per-kernel timing: the same steps again, each of the library's
+    # launches bracketed by CUDA events on its stream
+    per_kernel = {}
+    launches = None
+    kt_steps = 3
+    for i in range(kt_steps):
+        reset()
+        flush(i)
+        with abi.KernelTimer(max_launches=64) as kt:
+            step()
+        torch.cuda.synchronize()
+        launches = len(kt.names)
+        for kname, ms in kt.durations_ms():
+            per_kernel.setdefault(kname, []).append(ms)
+    per_kernel = merge_tails(per_kernel)
+
+    # ---- end to end through the ABI with host buffers
+    u_host = u.cpu().pin_memory()
+    X_host = X0.cpu().pin_memory()
+    out = X if residual else Y
+    Y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush(i)
+        ev2[i][0].record(stream)
+        u.copy_(u_host, non_blocking=True)
+        X.copy_(X_host, non_blocking=True)
+        step()
+        Y_host.copy_(out, non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2), world, device)
+
+    kernels = []
+    for kname, ms_list in per_kernel.items():
+        cnt = len(ms_list) / kt_steps
+        ms = statistics.mean(ms_list)
+        entry = {"kernel": kname, "launches_per_step": cnt, "ms": ms}
+        kw = prefill_kernel_work(kname, d, layers, sms, peaks, peak_kind)
+        if kw is not None:
+            bound, units, unit, peak, note = kw
+            scale = 1e12 if unit == "TFLOP/s" else 1e9
+            achieved = units / (ms / 1e3) / scale
+            entry.update({"bound": bound, "algorithmic_per_launch": units, "achieved": achieved,
+                          "peak": peak, "unit": unit, "frac": achieved / peak, "peak_note": note})
+        kernels.append(entry)
+    kernels.sort(key=lambda e: -e["ms"] * e["launches_per_step"])
+    dom = kernels[0]
+    roofline = {"bound": dom.get("bound"), "achieved": dom.get("achieved"), "peak": dom.get("peak"),
+                "unit": dom.get("unit"), "frac": dom.get("frac"),
+                "traffic": DRAM_TRAFFIC_EARLIER_CAPTURE.get(dom["kernel"]) if name == HEADLINE else None,
+                "traffic_note": "from an earlier ncu capture of this kernel on this workload (unchanged "
+                                "kernel), else null",
+                "kernel": dom["kernel"], "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
+    h2d = u.numel() * 2 + X0.numel() * 2
+    return {
+        "metric": METRICS[name], "value": value, "unit": UNIT, "ms_per_step": total_ms / steps,
+        "steps": steps, "config": config_of(name, d, layers, False),
+        "l2": "flushed between steps (256 MB write, then a 256 MB read of another buffer so no dirty lines "
+              "remain; outside the step events)",
+        "roofline": roofline, "kernels": kernels,
+        "e2e": {"value": world * steps * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": launches * steps,
+    }
 
 
-# --------------------------------------------------------------------- our arm
+# --------------------------------------------------------------------- our arm: decode
+
+def bench_decode(args, ctx, name):
+    import torch
+    from gated_memory_sharing_b200 import abi
+    from gated_memory_sharing_b200.layers import DecodeChain, GMULayer, ScanLayer
+    world, rank, device, flush, stream, peaks, peak_kind, sms = ctx
+    d, seed, layers, _ = workload_dims(name)
+    B, Di, Dm = d.batch, d.d_inner, d.d_model
+    w = synth.scan_weights(d, seed)
+    gws = [synth.gmu_weights(d, seed, layer=l) for l in range(layers)]
+    scan = ScanLayer(w, Dm, abi.BF16)
+    chain = DecodeChain(scan, [GMULayer(g["W1"], g["W2"], abi.BF16) for g in gws])
+    rs = seed + 7919 * rank
+    # the prompt (the workload's stated length), then a ring of per-step inputs
+    u0 = dev_normal((B, d.seqlen, Di), rs, device)
+    ring_u = dev_normal((DECODE_RING, B, Di), rs + 1, device)
+    ring_x = dev_normal((DECODE_RING, B, Dm), rs + 2, device)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    _, h, cs = scan.prefill(u0)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    prompt_ms = t0.elapsed_time(t1)
+    del u0
+    m = torch.empty(B, Di, dtype=torch.bfloat16, device=device)
+    x = torch.empty(B, Dm, dtype=torch.bfloat16, device=device)
+
+    def one(i):
+        x.copy_(ring_x[i % DECODE_RING])
+        chain.step(ring_u[i % DECODE_RING], h, cs, x, m_t=m)
+
+    for i in range(4):           # warm-up, workspaces, kernel attributes
+        one(i)
+    torch.cuda.synchronize()
+    # one step per graph (replayed with the L2 flushed before it), and a graph
+    # of 64 back-to-back steps
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1):
+        chain.step(ring_u[0], h, cs, x, m_t=m)
+    g64 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g64):
+        for i in range(64):
+            x.copy_(ring_x[i])
+            chain.step(ring_u[i], h, cs, x, m_t=m)
+    for _ in range(max(args.warmup, 3)):
+        g1.replay()
+        g64.replay()
+    torch.cuda.synchronize()
+    assert abi.sambay_device_status() == 0
+
+    # ---- headline: L2 flushed before every step (between two steps of this
+    # layer a model streams every other layer's weights through L2)
+    reps = max(args.steps, 20)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(reps):
+        flush(i)
+        ev[i][0].record(stream)
+        g1.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    step_us = 1e3 * total_ms / reps
+
+    # ---- the stated horizon back to back (graphs of 64 steps, no flush)
+    horizon = synth.DECODE_STEPS["decode_b64" if name == "decode_b64" else "sharing_b2_l8192"]
+    hz = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    torch.cuda.synchronize()
+    hz[0].record(stream)
+    for _ in range(horizon // 64):
+        g64.replay()
+    hz[1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    horizon_ms = max_over_ranks(hz[0].elapsed_time(hz[1]), world, device)
+
+    # ---- per-kernel breakdown of single steps (L2 flushed before each)
+    per_kernel = {}
+    launches = None
+    for i in range(4):
+        flush(i)
+        with abi.KernelTimer(max_launches=64) as kt:
+            chain.step(ring_u[i], h, cs, x, m_t=m)
+        torch.cuda.synchronize()
+        launches = len(kt.names)
+        for kname, ms in kt.durations_ms():
+            per_kernel.setdefault(kname, []).append(1e3 * ms)
+    kernels_us = {k: statistics.mean(v) for k, v in per_kernel.items()}
+
+    # ---- end to end: per step u_t and X from pinned host memory in, X (the
+    # layers' output) back out
+    u_host = ring_u[:64].cpu().pin_memory()
+    x_host = ring_x[:64].cpu().pin_memory()
+    y_host = torch.empty(64, B, Dm, dtype=torch.bfloat16).pin_memory()
+    u_dev = torch.empty(B, Di, dtype=torch.bfloat16, device=device)
+    e2e_steps = reps
+    ev2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    torch.cuda.synchronize()
+    ev2[0].record(stream)
+    for i in range(e2e_steps):
+        u_dev.copy_(u_host[i % 64], non_blocking=True)
+        x.copy_(x_host[i % 64], non_blocking=True)
+        chain.step(u_dev, h, cs, x, m_t=m)
+        y_host[i % 64].copy_(x, non_blocking=True)
+    ev2[1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(ev2[0].elapsed_time(ev2[1]), world, device)
+
+    nbytes = decode_bytes(d, B, layers)
+    achieved = nbytes / (step_us / 1e6) / 1e9
+    dom = max(kernels_us.items(), key=lambda kv: kv[1])
+    del g1, g64
+    return {
+        "metric": METRICS[name], "value": world * B / (step_us / 1e6), "unit": UNIT,
+        "us_per_step": step_us, "ms_per_step": step_us / 1e3, "steps": reps,
+        "config": config_of(name, d, layers, True),
+        "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the step events)",
+        "prompt_prefill_ms": prompt_ms,
+        "horizon": {"steps": horizon, "ms": horizon_ms, "us_per_step": 1e3 * horizon_ms / horizon,
+                    "note": "back-to-back steps in graphs of 64, L2 not flushed"},
+        "kernels_us": kernels_us,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_step": nbytes, "kernel": "whole decode step",
+                     "dominant_kernel": dom[0], "dominant_kernel_us": dom[1],
+                     "peak_note": f"{peak_kind} HBM copy"},
+        "e2e": {"value": world * e2e_steps * B / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": B * (Di + Dm) * 2, "d2h_bytes_per_step": B * Dm * 2},
+        "gpu_launches": launches * reps,
+    }
+
 
 def run_ours(args, world, rank, local):
     import torch
     from gated_memory_sharing_b200 import abi, build
-    from gated_memory_sharing_b200.layers import GMULayer, ScanLayer, to_device
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -289,153 +640,43 @@ def run_ours(args, world, rank, local):
     barrier(world)
     abi.load()
     peaks, peak_kind = load_peaks()
-
-    d, seed = synth.workload(WORKLOAD)
-    w = synth.scan_weights(d, seed)
-    gw = synth.gmu_weights(d, seed)
-    # each rank: its own sequence (weak scaling), the same weights
-    u_np = synth.scan_inputs(d, seed + 7919 * rank)
-    X_np = synth.gmu_inputs(d, seed + 7919 * rank)
-    scan = ScanLayer(w, d.d_model, abi.BF16)
-    gmu = GMULayer(gw["W1"], gw["W2"], abi.BF16)
-    u = to_device(u_np, abi.BF16)
-    X = to_device(X_np, abi.BF16)
-    T, Di, Dm = d.tokens, d.d_inner, d.d_model
-    M = torch.empty_like(u)
-    Y = torch.empty_like(X)
-    h, cs = scan.new_state(d.batch)
-    flush = L2Flush(device)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        scan.prefill(u, h, cs, M=M, fresh=True)
-
-    def gmu_step():
-        gmu.forward(X, M.view(T, Di), residual=False, Y=Y)
-
-    # warm-up (also sets kernel attributes outside the timed region)
-    for _ in range(max(args.warmup, 3)):
-        step()
-        gmu_step()
-    torch.cuda.synchronize()
-    assert abi.sambay_device_status() == 0
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    ctx = (world, rank, device, L2Flush(device), torch.cuda.current_stream(), peaks, peak_kind, sms)
+    names = [args.workload] if args.only_headline else \
+        [args.workload] + [n for n in WORKLOADS if n != args.workload]
 
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-
-    # ---- device-resident timed region: K steps, L2 flushed between steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush(i)
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-        gmu_step()
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    scan_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    gmu_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    step_ms = [a + b for a, b in zip(scan_ms, gmu_ms)]
-    total_ms = max_over_ranks(sum(step_ms), world, device)
-    value = world * args.steps * T / (total_ms / 1e3)
-
-    # ---- per-kernel timing: the same steps again, each of the library's
-    # launches bracketed by CUDA events on its stream
-    per_kernel = {}
-    launches_per_step = None
-    kt_steps = max(3, min(args.steps, 20))
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(kt_steps):
-        flush(i)
-        with abi.KernelTimer(max_launches=32) as kt:
-            step()
-            gmu_step()
+    results = {}
+    for name in names:
+        fn = bench_decode if workload_dims(name)[3] else bench_prefill
+        results[name] = fn(args, ctx, name)
         torch.cuda.synchronize()
-        launches_per_step = len(kt.names)
-        for name, ms in kt.durations_ms():
-            per_kernel.setdefault(name, []).append(ms)
-    barrier(world)
-
-    # ---- end to end through the ABI with host buffers
-    u_host = u.cpu().pin_memory()
-    X_host = X.cpu().pin_memory()
-    Y_host = torch.empty(Y.shape, dtype=Y.dtype).pin_memory()
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush(i)
-        ev2[i][0].record(stream)
-        u.copy_(u_host, non_blocking=True)
-        X.copy_(X_host, non_blocking=True)
-        step()
-        gmu_step()
-        Y_host.copy_(Y, non_blocking=True)
-        ev2[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(args.steps)),
-                            world, device)
-    e2e_value = world * args.steps * T / (e2e_ms / 1e3)
-
-    # ---- decode sub-benchmark: 64 sequences, one token each per step
-    decode = None
-    if not args.no_decode:
-        decode = bench_decode(args, scan, gmu, d, seed + 7919 * rank, flush, stream, world, device, peaks)
+        assert abi.sambay_device_status() == 0, f"device status after {name}"
     clk = clocks.stop()
-    assert abi.sambay_device_status() == 0
 
-    # ---- roofline of every kernel; the dominant one (longest per step) leads
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    kernels = []
-    for name, ms_list in per_kernel.items():
-        launches = len(ms_list) / kt_steps
-        ms = statistics.mean(ms_list)
-        entry = {"kernel": name, "launches_per_step": launches, "ms": ms}
-        kw = kernel_work(name, d, sms, peaks, peak_kind)
-        if kw is not None:
-            bound, units, unit, peak, peak_note = kw
-            scale = 1e12 if unit == "TFLOP/s" else 1e9
-            achieved = units / (ms / 1e3) / scale
-            entry.update({"bound": bound, "algorithmic_per_launch": units, "achieved": achieved,
-                          "peak": peak, "unit": unit, "frac": achieved / peak, "peak_note": peak_note})
-        kernels.append(entry)
-    kernels.sort(key=lambda e: -e["ms"] * e["launches_per_step"])
-    dom = kernels[0]
-    roofline = {"bound": dom.get("bound"), "achieved": dom.get("achieved"), "peak": dom.get("peak"),
-                "unit": dom.get("unit"), "frac": dom.get("frac"),
-                "traffic": DRAM_TRAFFIC.get(dom["kernel"]), "kernel": dom["kernel"],
-                "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
-    scan_mean_ms = statistics.mean(scan_ms)
-    gmu_mean_ms = statistics.mean(gmu_ms)
-
+    head = results[args.workload]
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": d.batch, "seq_len": d.seqlen,
-                   "d_model": Dm, "d_inner": Di, "d_state": d.d_state, "d_conv": d.d_conv,
-                   "dt_rank": d.dt_rank, "gmu_layers": 1, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between steps (256 MB write, then a 256 MB read of another buffer so no "
-                         "dirty lines remain; outside the step events)"},
-        "roofline": roofline,
-        "breakdown_ms": {"scan_prefill": scan_mean_ms, "gmu_forward": gmu_mean_ms},
-        "kernels": kernels,
-        "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": u.numel() * 2 + X.numel() * 2,
-                "d2h_bytes_per_step": Y.numel() * 2},
-        "gpu_launches": launches_per_step * args.steps,   # counted by the library's launch hook
+        "metric": head["metric"], "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(head["config"], parallelism=f"replicas x{world}", l2=head["l2"]),
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": clk,
+        "peaks": peak_kind,
     }
-    if decode is not None:
-        out["decode"] = decode
+    for k in ("kernels", "kernels_us", "horizon", "prompt_prefill_ms", "us_per_step"):
+        if k in head:
+            out[k] = head[k]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_oracle()
+        for name in names:
+            results[name]["cpu_baseline"] = cpu_baseline(name)
+        out["cpu_baseline"] = results[args.workload]["cpu_baseline"]
+    out["workloads"] = {n: r for n, r in results.items() if n != args.workload}
     if rank == 0:
         print(json.dumps(out), flush=True)
     barrier(world)
@@ -443,84 +684,14 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
-def bench_decode(args, scan, gmu, d, seed, flush, stream, world, device, peaks):
-    import torch
-    from gated_memory_sharing_b200.layers import to_device
-    B, Di, Dm = DECODE_BATCH, d.d_inner, d.d_model
-    dd = synth.Dims(B, 16, Dm, Di, d.d_state, d.d_conv, d.dt_rank, synth.BF16)
-    u0 = to_device(synth.scan_inputs(dd, seed + 1), 1)                       # 16-token prompt
-    ring_u = to_device(synth.scan_inputs(dd, seed + 2, seqlen=DECODE_RING, tag="u_dec"), 1)
-    ring_x = to_device(synth.gmu_inputs(dd, seed + 3, rows=B * DECODE_RING, tag="X_dec"), 1)
-    ring_u = ring_u.transpose(0, 1).contiguous()                              # [ring, B, Di]
-    ring_x = ring_x.view(DECODE_RING, B, Dm)
-    _, h, cs = scan.prefill(u0)
-    m = torch.empty(B, Di, dtype=torch.bfloat16, device=device)
-    y = torch.empty(DECODE_RING, B, Dm, dtype=torch.bfloat16, device=device)
-
-    def steps():
-        for i in range(DECODE_RING):
-            scan.step(ring_u[i], h, cs, m_t=m)
-            gmu.step(ring_x[i], m, residual=True, Y=y[i])
-
-    steps()                      # warm-up, workspaces, kernel attributes
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        steps()
-    for _ in range(max(args.warmup, 3)):
-        g.replay()
-    torch.cuda.synchronize()
-    reps = max(args.steps // 4, 5)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(reps):
-        flush(i)
-        ev[i][0].record(stream)
-        g.replay()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
-    step_us = 1e3 * total_ms / (reps * DECODE_RING)
-    # per-kernel breakdown of a few eager steps (launch gaps excluded)
-    from gated_memory_sharing_b200 import abi
-    per_kernel = {}
-    for i in range(4):
-        with abi.KernelTimer(max_launches=32) as kt:
-            scan.step(ring_u[i], h, cs, m_t=m)
-            gmu.step(ring_x[i], m, residual=True, Y=y[i])
-        torch.cuda.synchronize()
-        for name, ms in kt.durations_ms():
-            per_kernel.setdefault(name, []).append(1e3 * ms)
-    kernels_us = {k: statistics.mean(v) for k, v in per_kernel.items()}
-    # algorithmic bytes per decode step (every byte the step must move once)
-    state = B * Di * d.d_state * 4 * 2 + B * Di * d.d_conv * 2 * 2
-    weights = (d.dt_rank + 2 * d.d_state) * Di * 2 + Di * d.dt_rank * 2 + Di * (d.d_conv + 1) * 2 \
-        + Di * d.d_state * 4 + 2 * Di * 4 + 2 * Di * Dm * 2
-    acts = B * (2 * Di + 3 * Dm) * 2
-    nbytes = state + weights + acts
-    achieved = nbytes / (step_us / 1e6) / 1e9
-    del g
-    return {"metric": "decode tokens/s (scan step + GMU step)", "unit": UNIT,
-            "value": world * B / (step_us / 1e6), "us_per_step": step_us, "batch": B,
-            "steps_timed": reps * DECODE_RING,
-            "setup": "16-token prompt prefill; the decode state has a fixed size, so the step "
-                     "cost does not depend on the position",
-            "l2": "flushed between graph replays of 64 back-to-back steps (256 MB write + 256 MB read)",
-            "kernels_us": kernels_us,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "algorithmic_bytes_per_step": nbytes}}
-
-
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--workload", choices=WORKLOADS, default=HEADLINE)
+    ap.add_argument("--only-headline", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

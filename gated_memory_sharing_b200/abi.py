@@ -38,6 +38,9 @@ EXPORTS = (
     "sambay_scan_step_noalloc",
     "gmu_forward",
     "gmu_step",
+    "sambay_decode_step_workspace",
+    "sambay_decode_step",
+    "sambay_gmu_step_stall_test",
     "sambay_profile_begin",
     "sambay_profile_end",
     "sambay_device_status",
@@ -77,6 +80,13 @@ class ScanWeights(ctypes.Structure):
     ]
 
 
+class GmuWeights(ctypes.Structure):
+    _fields_ = [
+        ("W1", ctypes.c_void_p),
+        ("W2", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -92,6 +102,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
     pd, pw = ctypes.POINTER(Dims), ctypes.POINTER(ScanWeights)
+    pg = ctypes.POINTER(GmuWeights)
     sig = {
         "sambay_scan_prefill_workspace": (sz, [pd]),
         "sambay_scan_step_workspace": (sz, [pd]),
@@ -102,6 +113,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sambay_scan_step_noalloc": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp]),
         "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sambay_decode_step_workspace": (sz, [pd, i32]),
+        "sambay_decode_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, i32, pg, vp, vp, sz, vp]),
+        "sambay_gmu_step_stall_test": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                      ctypes.c_uint64, vp]),
         "sambay_profile_begin": (ctypes.c_int, [ctypes.POINTER(vp), i32]),
         "sambay_profile_end": (i32, [ctypes.POINTER(ctypes.c_char_p), i32]),
         "sambay_device_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
@@ -175,6 +190,36 @@ def sambay_scan_step(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv
     _check("sambay_scan_step", load().sambay_scan_step(
         ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state),
         _p(conv_state), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_decode_step_workspace(dims: Dims, n_layers: int) -> int:
+    return load().sambay_decode_step_workspace(ctypes.byref(dims), n_layers)
+
+
+def make_gmu_layers(pairs):
+    """Host array of GmuWeights from (W1, W2) tensor pairs."""
+    arr = (GmuWeights * max(1, len(pairs)))()
+    for i, (w1, w2) in enumerate(pairs):
+        arr[i] = GmuWeights(w1.data_ptr(), w2.data_ptr())
+    return arr
+
+
+def sambay_decode_step(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv_state, layers,
+                       n_layers: int, X, ws, stream=None):
+    """One decode token: scan step, then X <- X + GMU_l(X, m_t) for each layer
+    (``layers``: the array make_gmu_layers returns)."""
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_decode_step", load().sambay_decode_step(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state), _p(conv_state),
+        n_layers, layers, _p(X), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_gmu_step_stall_test(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws,
+                               wait_limit_cycles: int, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_gmu_step_stall_test", load().sambay_gmu_step_stall_test(
+        ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(residual), _p(Y), _p(ws),
+        ws_bytes, wait_limit_cycles, _stream(stream)))
 
 
 # Library-owned scratch size of sambay_scan_step_noalloc (bytes, per GPU).

@@ -1,11 +1,12 @@
 // libsambay: C ABI of the SambaY scan + Gated Memory Unit hot path on B200.
 // Host side: argument validation, workspace carving, TMA descriptors and
 // kernel launches.  Every step of the computation runs in the kernels of
-// scan_kernels.cuh, tc_gemm.cuh and simt_gemm.cuh.
+// scan_kernels.cuh, step_kernels.cuh, tc_gemm.cuh and simt_gemm.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <vector>
@@ -14,6 +15,7 @@
 #include "common.cuh"
 #include "scan_kernels.cuh"
 #include "simt_gemm.cuh"
+#include "step_kernels.cuh"
 #include "tc_gemm.cuh"
 
 using sambay::bf16;
@@ -162,13 +164,70 @@ int xproj_splits(long long rows, int d_inner) {
 // dt_rank rounded up to whole 64-wide K blocks (each half of the split delta)
 int rank_pad(int R) { return (R + 63) / 64 * 64; }
 
+// The bf16 decode step (step_kernels.cuh): the channels are cut into slices of
+// `chan` (a multiple of 8, at most kMaxChan) with about one slice per SM of a
+// 148-SM B200 (a function of the sizes only, so the workspace and the
+// summation order do not depend on the device), and each CTA takes up to
+// `group` sequences of its slice.
+constexpr int kMaxDynSmemBytes = 232448;
+
+struct StepPlan {
+  bool ok = false;
+  int chan = 0, nslice = 0, group = 0, Rp = 0;
+  size_t smem = 0;
+};
+
+StepPlan step_plan(const sambay_dims* d) {
+  StepPlan sp;
+  if (d->io != SAMBAY_BF16) return sp;
+  const int Di = d->d_inner;
+  for (int c = 8; c <= sambay::step::kMaxChan; c += 8)
+    if (Di % c == 0 && Di / c <= kSplitTarget) { sp.chan = c; break; }
+  if (sp.chan == 0) return sp;                    // wider than 148 slices of 48 channels
+  sp.nslice = Di / sp.chan;
+  sp.Rp = (d->dt_rank + 15) / 16 * 16;
+  int group = std::min(d->batch, sambay::step::kMaxGroup);
+  while (group > 4 && sambay::step::ScanStepLayout(sp.chan, group, sp.Rp).bytes > kMaxDynSmemBytes) group -= 4;
+  const sambay::step::ScanStepLayout ly(sp.chan, group, sp.Rp);
+  if (ly.bytes > kMaxDynSmemBytes) return sp;
+  sp.group = group;
+  sp.smem = static_cast<size_t>(ly.bytes);
+  sp.ok = true;
+  return sp;
+}
+
 struct ScanWs {
   size_t uc, part, xdbl, delta, dt, bcp, total;
   int splits;
 };
 
-ScanWs scan_ws_layout(const sambay_dims* d, long long T) {
+// Scratch of the bf16 decode step: conv output, x_proj partials per slice,
+// the split delta and B | C.
+struct StepWs {
+  size_t uc, part, dts, bc, total;
+};
+
+StepWs step_ws_layout(const sambay_dims* d, const StepPlan& sp) {
+  StepWs w{};
+  const size_t B = d->batch, Di = d->d_inner, ldx = d->dt_rank + 2 * d->d_state;
+  size_t off = 0;
+  w.uc = off;   off += round256(B * Di * 4);
+  w.part = off; off += round256(static_cast<size_t>(sp.nslice) * ldx * B * 4);
+  w.dts = off;  off += round256(2 * B * static_cast<size_t>(sp.Rp) * 2);
+  w.bc = off;   off += round256(B * 2 * d->d_state * 4);
+  w.total = off;
+  return w;
+}
+
+ScanWs scan_ws_layout(const sambay_dims* d, long long T, bool step = false) {
   ScanWs w{};
+  if (step) {
+    const StepPlan sp = step_plan(d);
+    if (sp.ok) {
+      w.total = step_ws_layout(d, sp).total;
+      return w;
+    }
+  }
   const long long Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
   const bool tc = d->io == SAMBAY_BF16;
   w.splits = tc ? xproj_splits(T, d->d_inner) : 1;
@@ -724,11 +783,71 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
   return SAMBAY_OK;
 }
 
+sambay_status scan_step_fused(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
+                              const StepPlan& sp, const void* u_t, void* m_t, float* ssm_state,
+                              void* conv_state, uint8_t* ws, cudaStream_t st) {
+  auto kproj = sambay::step::step_proj_kernel;
+  auto kred = sambay::step::step_reduce_kernel;
+  auto kscan = sambay::step::step_scan_kernel;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kscan, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmemBytes) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  SAMBAY_MAX_CARVEOUT(kproj, dev);
+  SAMBAY_MAX_CARVEOUT(kred, dev);
+  SAMBAY_MAX_CARVEOUT(kscan, dev);
+  const StepWs L = step_ws_layout(d, sp);
+  sambay::step::StepParams p{};
+  p.u_t = static_cast<const bf16*>(u_t);
+  p.conv_state = static_cast<bf16*>(conv_state);
+  p.conv_w = static_cast<const bf16*>(w->conv_w);
+  p.conv_b = static_cast<const bf16*>(w->conv_b);
+  p.x_proj_w = static_cast<const bf16*>(w->x_proj_w);
+  p.dt_proj_w = static_cast<const bf16*>(w->dt_proj_w);
+  p.dt_bias = w->dt_bias;
+  p.A = w->A;
+  p.D = w->D;
+  p.h = ssm_state;
+  p.m_t = static_cast<bf16*>(m_t);
+  p.uc = reinterpret_cast<float*>(ws + L.uc);
+  p.part = reinterpret_cast<float*>(ws + L.part);
+  p.dts = reinterpret_cast<bf16*>(ws + L.dts);
+  p.bc = reinterpret_cast<float*>(ws + L.bc);
+  p.B = d->batch;
+  p.Di = d->d_inner;
+  p.R = d->dt_rank;
+  p.Rp = sp.Rp;
+  p.ldx = d->dt_rank + 2 * d->d_state;
+  p.chan = sp.chan;
+  p.nslice = sp.nslice;
+  p.group = sp.group;
+  const dim3 grid(sp.nslice, (d->batch + sp.group - 1) / sp.group);
+  const dim3 block(sambay::step::kThreads);
+  {
+    ProfScope ps("step_proj", st);
+    if (launch_k(kproj, grid, block, 0, st, false, 1, p) != cudaSuccess) return SAMBAY_ERR_CUDA;
+  }
+  {
+    const long long outs = static_cast<long long>(p.ldx) * p.B * sambay::step::kRedLanes;
+    ProfScope ps("step_reduce", st);
+    if (launch_k(kred, dim3(grid_for(outs, sambay::step::kThreads, sms)), block, 0, st, true, 1, p) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+  }
+  ProfScope ps("step_scan", st);
+  return launch_k(kscan, grid, block, sp.smem, st, true, 1, p) == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+}
+
 template <typename T>
 sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
                              const void* u_t, void* m_t, float* ssm_state, void* conv_state,
                              uint8_t* ws, cudaStream_t st) {
   const long long B = d->batch;
+  if (sizeof(T) == 2) {
+    const StepPlan sp = step_plan(d);
+    if (sp.ok) return scan_step_fused(dev, sms, w, d, sp, u_t, m_t, ssm_state, conv_state, ws, st);
+  }
   const ScanWs L = scan_ws_layout(d, B);
   T* uc = reinterpret_cast<T*>(ws + L.uc);
   constexpr int VEC = 16 / sizeof(T);
@@ -782,6 +901,49 @@ sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* 
   return SAMBAY_OK;
 }
 
+// How a decode GMU layer's kernels chain onto the work before them.
+struct StepChain {
+  bool chained = false;      // the gate GEMM follows a kernel of this call (PDL)
+  bool x_independent = false;  // ... which does not write X: the whole gate main loop may start early
+  unsigned long long wait_limit = 0;
+  int stall_test = 0;
+};
+
+// Decode GMU, bf16: H^T = SiLU(W1 X^T) ⊙ M^T, then Y^T = W2^T H^T (+ residual^T)
+// as swap-AB tensor-core GEMMs whose weights are the A operand and stream
+// once.  Split-K over clusters of CTAs (csplit): each split keeps its partial
+// tile in shared memory; after a cluster barrier each CTA sums a slice of the
+// tile's rows over the cluster (distributed shared memory).  The out GEMM is
+// launched with programmatic dependent launch and loads its first W2 tiles
+// before waiting for the gate GEMM.
+sambay_status gmu_step_tc(int dev, int sms, const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                          const void* W1, const void* W2, const void* residual, void* Y, uint8_t* Hbuf,
+                          const StepChain& ch, cudaStream_t st) {
+  const int Dm = d->d_model, Di = d->d_inner, Bn = static_cast<int>(rows);
+  bf16* H = reinterpret_cast<bf16*>(Hbuf);
+  auto g1 = tc_args(Di, Bn, Dm, H, Di, M);
+  auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual);
+  g1.csplit = g2.csplit = 1;
+  g1.a_early = ch.chained ? 1 : 0;
+  g1.b_early = (ch.chained && ch.x_independent) ? 1 : 0;
+  g2.a_early = 1;
+  g1.wait_limit = g2.wait_limit = ch.wait_limit;
+  g1.stall_test = g2.stall_test = ch.stall_test;
+  const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
+#define SAMBAY_STEP_GEMMS(BNV)                                                                              \
+  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1,   \
+                                                                    kStepMaxSplits, st, ch.chained)));       \
+  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2,    \
+                                                                    kStepMaxSplits, st, true)));
+  if (Bn <= 32) { SAMBAY_STEP_GEMMS(32) }
+  else if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
+  else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
+  else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }
+  else { SAMBAY_STEP_GEMMS(256) }
+#undef SAMBAY_STEP_GEMMS
+  return SAMBAY_OK;
+}
+
 }  // namespace
 
 // Scratch of sambay_scan_step_noalloc: a fixed array compiled into the
@@ -792,7 +954,9 @@ sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SAMBAY_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+// device address of g_noalloc_scratch, per device; host threads racing on a
+// device's first call both store the same value
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
 }  // namespace
 
 // ====================================================================== C ABI
@@ -824,7 +988,7 @@ size_t sambay_scan_step_workspace(const sambay_dims* d) {
   sambay_dims e = *d;
   e.seqlen = 1;
   if (check_dims(&e, false, true) != SAMBAY_OK) return 0;
-  return scan_ws_layout(&e, e.batch).total;
+  return scan_ws_layout(&e, e.batch, true).total;
 }
 
 size_t gmu_forward_workspace(const sambay_dims* d, int64_t rows) {
@@ -913,25 +1077,83 @@ sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, residual, Y, w8, L, st);
-  const int Dm = d->d_model, Di = d->d_inner, Bn = static_cast<int>(rows);
-  bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
-  // swap-AB: H^T = SiLU(W1 X^T) ⊙ M^T; W1 rows stream once through the tensor
-  // cores.  Split-K over clusters of CTAs (csplit): each split keeps its
-  // partial tile in shared memory; after a cluster barrier each CTA sums a
-  // slice of the tile's rows over the cluster (distributed shared memory).
-  auto g1 = tc_args(Di, Bn, Dm, H, Di, M);
-  auto g2 = tc_args(Dm, Bn, Di, Y, Dm, residual);
-  g1.csplit = g2.csplit = 1;
-  const Operand w1{W1, Di, Dm}, xr{X, rows, Dm}, w2{W2, Di, Dm}, hr{H, rows, Di};
-#define SAMBAY_STEP_GEMMS(BNV)                                                                   \
-  SAMBAY_TRY((run_tc<BNV, false, false, sambay::tc::EPI_GATE, true>("gmu_step_gate", dev, sms, w1, xr, g1, kStepMaxSplits, st, false))); \
-  SAMBAY_TRY((run_tc<BNV, true, false, sambay::tc::EPI_RESID, true>("gmu_step_out", dev, sms, w2, hr, g2, kStepMaxSplits, st, true)));
-  if (Bn <= 64) { SAMBAY_STEP_GEMMS(64) }
-  else if (Bn <= 128) { SAMBAY_STEP_GEMMS(128) }
-  else if (Bn <= 192) { SAMBAY_STEP_GEMMS(192) }
-  else { SAMBAY_STEP_GEMMS(256) }
-#undef SAMBAY_STEP_GEMMS
+  return gmu_step_tc(dev, sms, d, rows, X, M, W1, W2, residual, Y, w8 + L.h, StepChain{}, st);
+}
+
+size_t sambay_decode_step_workspace(const sambay_dims* d, int32_t n_layers) {
+  if (!d || n_layers < 0) return 0;
+  sambay_dims e = *d;
+  e.seqlen = 1;
+  if (check_dims(&e, true, true) != SAMBAY_OK || e.batch > kStepMaxRows) return 0;
+  const size_t scan = scan_ws_layout(&e, e.batch, true).total;
+  const size_t gmu = n_layers > 0 ? gmu_ws_layout(&e, e.batch, true).total : 0;
+  return round256(scan) + gmu;
+}
+
+sambay_status sambay_decode_step(const sambay_scan_weights* w, const sambay_dims* d, const void* u_t,
+                                 void* m_t, float* ssm_state, void* conv_state, int32_t n_layers,
+                                 const sambay_gmu_weights* layers, void* X, void* ws, size_t ws_bytes,
+                                 sambay_stream_t stream) {
+  if (!d) return SAMBAY_ERR_INVALID_ARG;
+  sambay_dims e = *d;
+  e.seqlen = 1;
+  SAMBAY_TRY(check_dims(&e, true, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u_t, m_t, ssm_state, conv_state}));
+  if (m_t == u_t) return SAMBAY_ERR_INVALID_ARG;
+  if (n_layers < 0 || n_layers > 1024) return SAMBAY_ERR_INVALID_ARG;
+  if (e.batch > kStepMaxRows) return SAMBAY_ERR_UNSUPPORTED;
+  if (n_layers > 0) {
+    if (!layers) return SAMBAY_ERR_INVALID_ARG;
+    SAMBAY_TRY(check_ptrs({X}));
+    for (int l = 0; l < n_layers; ++l) SAMBAY_TRY(check_ptrs({layers[l].W1, layers[l].W2}));
+    if (X == m_t || X == u_t) return SAMBAY_ERR_INVALID_ARG;
+  }
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_decode_step_workspace(&e, n_layers)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (e.io == SAMBAY_BF16) {
+    SAMBAY_TRY(scan_step_impl<bf16>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st));
+  } else {
+    SAMBAY_TRY(scan_step_impl<float>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st));
+  }
+  const GmuWs L = gmu_ws_layout(&e, e.batch, true);
+  uint8_t* gw8 = w8 + round256(scan_ws_layout(&e, e.batch, true).total);   // H, after the scan scratch
+  for (int l = 0; l < n_layers; ++l) {
+    if (e.io == SAMBAY_F32) {
+      SAMBAY_TRY(gmu_f32(&e, e.batch, X, m_t, layers[l].W1, layers[l].W2, X, X, gw8, L, st));
+      continue;
+    }
+    // layer 0's gate reads the caller's X, untouched by the scan step, so its
+    // whole main loop may overlap the scan; later gates read the X the layer
+    // before wrote and load only their W1 tiles early
+    StepChain ch;
+    ch.chained = true;
+    ch.x_independent = (l == 0);
+    SAMBAY_TRY(gmu_step_tc(dev, sms, &e, e.batch, X, m_t, layers[l].W1, layers[l].W2, X, X, gw8 + L.h, ch, st));
+  }
   return SAMBAY_OK;
+}
+
+sambay_status sambay_gmu_step_stall_test(const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                                         const void* W1, const void* W2, const void* residual, void* Y,
+                                         void* ws, size_t ws_bytes, uint64_t wait_limit_cycles,
+                                         sambay_stream_t stream) {
+  SAMBAY_TRY(gmu_common_checks(d, rows, X, M, W1, W2, residual, Y));
+  if (d->io != SAMBAY_BF16) return SAMBAY_ERR_UNSUPPORTED;
+  if (rows > kStepMaxRows) return SAMBAY_ERR_UNSUPPORTED;
+  if (wait_limit_cycles < 1 || wait_limit_cycles > (1ull << 32)) return SAMBAY_ERR_INVALID_ARG;
+  const GmuWs L = gmu_ws_layout(d, rows, true);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  StepChain ch;
+  ch.wait_limit = wait_limit_cycles;
+  ch.stall_test = 1;
+  return gmu_step_tc(dev, sms, d, rows, X, M, W1, W2, residual, Y, static_cast<uint8_t*>(ws) + L.h, ch,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const sambay_dims* d,
@@ -947,15 +1169,15 @@ sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const samba
   if (sambay_scan_step_workspace(&e) > SAMBAY_NOALLOC_SCRATCH_BYTES) return SAMBAY_ERR_UNSUPPORTED;
   int dev, sms;
   SAMBAY_TRY(current_device(&dev, &sms));
-  if (g_noalloc_ptr[dev] == nullptr) {
+  void* scratch = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {
     // once per device, with that device current
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr)
       return SAMBAY_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    g_noalloc_ptr[dev].store(scratch, std::memory_order_release);
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* w8 = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  uint8_t* w8 = static_cast<uint8_t*>(scratch);
   if (e.io == SAMBAY_BF16)
     return scan_step_impl<bf16>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);
   return scan_step_impl<float>(dev, sms, w, &e, u_t, m_t, ssm_state, conv_state, w8, st);

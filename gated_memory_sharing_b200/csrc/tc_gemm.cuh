@@ -332,6 +332,14 @@ struct GemmArgs {
   int tail_kbps;      // tail_ksplit units of tail_kbps k-blocks, each writing its fp32
   float* tail_part;   // partial tile [tail tile][split][tile rows][BN] to tail_part;
                       // tail_reduce_kernel sums them and applies the epilogue
+  int a_early;        // launched with programmatic dependent launch: the A operand does
+                      // not depend on the kernel before this one, so the producer loads
+                      // the first pipeline stages' A tiles before griddepcontrol.wait
+  int b_early;        // ... and neither does B: the whole main loop may run before the
+                      // wait; only the epilogue (aux in, output out) waits
+  unsigned long long wait_limit;  // bounded-wait limit in clock64 cycles (0: kWaitCycles)
+  int stall_test;     // fault-detector test: the epilogue first waits on a barrier that
+                      // nothing arrives at, so that wait runs out after wait_limit
 };
 
 // The final op on one element.  `o` is the output's linear index, `a` the aux
@@ -487,11 +495,19 @@ struct Cfg {
   static constexpr int kHalves = EW / 4;
   static constexpr bool kTmaEpi = !TRANS && (KIND == EPI_GATE || KIND == EPI_RESID || KIND == EPI_SOFTPLUS);
   static constexpr int kSlots = !kTmaEpi ? 0 : (KIND == EPI_SOFTPLUS ? 2 * kHalves : BN / 64);
-  static constexpr int kStageArea = kSlots * kSlotBytes > EW * kEpiWarpBytes ? kSlots * kSlotBytes : EW * kEpiWarpBytes;
+  // TRANS (swap-AB decode): the element-wise epilogue needs no staging; the area
+  // holds the aux of the cluster split-K reduction: for each of the BN output
+  // columns, the 8-aligned run of tile rows around the CTA's reduction rows
+  // (at most BM / 2 + 14 rows, since splits >= 2), at a pitch of kAuxPitch
+  static constexpr int kAuxPitch = 80;
+  static constexpr int kStageArea = TRANS ? BN * kAuxPitch * 2
+                                          : (kSlots * kSlotBytes > EW * kEpiWarpBytes ? kSlots * kSlotBytes
+                                                                                     : EW * kEpiWarpBytes);
   static constexpr int kEpiBytes = kStageArea + (kTmaEpi ? 1024 /*bias*/ : 0);
   static constexpr int kFixed = 1024 /*align slack*/ + 512 /*barriers*/ + kEpiBytes;
   static constexpr int kStagesFit = (kMaxDynSmem - kFixed) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kStageCap = 8;
+  static constexpr int kStages = kStagesFit > kStageCap ? kStageCap : kStagesFit;
   static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t kIdesc = idesc_bf16(kBMT, BN, A_MN, B_MN);
@@ -504,6 +520,7 @@ struct Cfg {
   static_assert(kSmem <= kMaxDynSmem, "shared memory budget");
   static_assert(EW == 4 || EW == 8, "one or two epilogue warps per TMEM lane quarter");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, whole 32-column epilogue chunks");
+  static_assert(!TRANS || EW == 4, "decode epilogue: one warp per TMEM lane quarter");
   static_assert(!B_MN || kBHalf % 64 == 0, "MN-major B tiles are whole 64-element atoms");
   static_assert(!PAIR || (!TRANS && !A_MN && KIND != EPI_F32_PARTIAL), "pairs serve the row-major prefill GEMMs");
 };
@@ -637,9 +654,12 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const unsigned long long wl = g.wait_limit ? g.wait_limit : kWaitCycles;
   // the set-up above touched only this CTA's shared memory and TMEM; global
-  // reads and writes wait for the kernel before this one on the stream
-  pdl_wait();
+  // reads and writes wait for the kernel before this one on the stream,
+  // except the producer's loads of operands flagged independent of it
+  // (a_early / b_early), which it orders itself
+  if (warp != 0 || !(g.a_early || g.b_early)) pdl_wait();
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -649,34 +669,63 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;  // per stage: outstanding load, its parity
       bool ok = true;
+      // a_early: the A tiles of the first S k-blocks (stages that are free from
+      // the start) are issued before griddepcontrol.wait, their B tiles after it
+      int n_early = 0;
+      const bool split_wait = g.a_early && !g.b_early;
+      auto load = [&](void* dst, const CUtensorMap* map, int st, int c0, int c1) {
+        if (PAIR) tma_load_2d_pair(dst, map, &full[st], c0, c1);
+        else tma_load_2d(dst, map, &full[st], c0, c1);
+      };
+      auto load_a = [&](int st, int arow, int kb) {
+        uint8_t* a_dst = sA + st * C::kABytes;
+        if (A_MN) {  // [K, M] in memory: boxes of 64 m x 64 k
+          load(a_dst, &tmA, st, arow, kb * BK);
+          load(a_dst + 8192, &tmA, st, arow + 64, kb * BK);
+        } else {     // [M, K]: one box of 64 k x 128 m
+          load(a_dst, &tmA, st, kb * BK, arow);
+        }
+      };
+      auto load_b = [&](int st, int hb, int bcol, int kb) {
+        uint8_t* b_dst = sB + st * C::kBBytes;
+        const int kb_b = g.b_k_wrap > 0 ? (kb * BK) % g.b_k_wrap : kb * BK;
+        if (B_MN) {  // [K, N]: boxes of 64 n x 64 k
+#pragma unroll
+          for (int j = 0; j < C::kBHalf / 64; ++j)
+            if (64 * j < hb) load(b_dst + j * 8192, &tmB, st, bcol + 64 * j, kb_b);
+        } else {     // [N, K]: one box of 64 k x kBHalf n (tail units: 64 k x hb n)
+          load(b_dst, hb == C::kBHalf ? &tmB : &tmB2, st, kb_b, bcol);
+        }
+      };
+      if (split_wait) {
+        for (int t = unit0; t < g.tiles && n_early < S; t += ustride) {
+          const TileCoord c = tile_coord<BN>(g, t);
+          const int hb = PAIR ? c.bn / 2 : c.bn;
+          for (int kb = c.kb0; kb < c.kb1 && n_early < S; ++kb, ++n_early) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[n_early], (C::kABytes + hb * BK * 2) * (PAIR ? 2 : 1));
+            load_a(n_early, c.m * C::kBMT + rank * BM, kb);
+          }
+        }
+      }
+      // a_early: wait before the first B tile; b_early: every operand is
+      // independent of the previous kernel and the producer never waits
+      if (split_wait) pdl_wait();
+      int item = 0;                   // position in this CTA's (tile, k-block) sequence
       for (int t = unit0; t < g.tiles && ok; t += ustride) {
         const TileCoord c = tile_coord<BN>(g, t);
         const int arow = c.m * C::kBMT + rank * BM;       // this CTA's A rows
         const int hb = PAIR ? c.bn / 2 : c.bn;            // this CTA's B columns
         const int bcol = c.n0 + rank * hb;
-        for (int kb = c.kb0; kb < c.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          // the leader's barrier counts the bytes of both CTAs of a pair
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], (C::kABytes + hb * BK * 2) * (PAIR ? 2 : 1));
-          uint8_t* a_dst = sA + stage * C::kABytes;
-          uint8_t* b_dst = sB + stage * C::kBBytes;
-          auto load = [&](void* dst, const CUtensorMap* map, int c0, int c1) {
-            if (PAIR) tma_load_2d_pair(dst, map, &full[stage], c0, c1);
-            else tma_load_2d(dst, map, &full[stage], c0, c1);
-          };
-          if (A_MN) {  // [K, M] in memory: boxes of 64 m x 64 k
-            load(a_dst, &tmA, arow, kb * BK);
-            load(a_dst + 8192, &tmA, arow + 64, kb * BK);
-          } else {     // [M, K]: one box of 64 k x 128 m
-            load(a_dst, &tmA, kb * BK, arow);
-          }
-          const int kb_b = g.b_k_wrap > 0 ? (kb * BK) % g.b_k_wrap : kb * BK;
-          if (B_MN) {  // [K, N]: boxes of 64 n x 64 k
-#pragma unroll
-            for (int j = 0; j < C::kBHalf / 64; ++j)
-              if (64 * j < hb) load(b_dst + j * 8192, &tmB, bcol + 64 * j, kb_b);
-          } else {     // [N, K]: one box of 64 k x kBHalf n (tail units: 64 k x hb n)
-            load(b_dst, hb == C::kBHalf ? &tmB : &tmB2, kb_b, bcol);
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++item) {
+          if (item < n_early) {
+            // A already issued and the barrier armed: the B half only (stage == item)
+            load_b(stage, hb, bcol, kb);
+          } else {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, wl)) { ok = false; break; }
+            // the leader's barrier counts the bytes of both CTAs of a pair
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], (C::kABytes + hb * BK * 2) * (PAIR ? 2 : 1));
+            load_a(stage, arow, kb);
+            load_b(stage, hb, bcol, kb);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -704,12 +753,12 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       bool ok = true;
       for (int t = unit0; t < g.tiles && ok; t += ustride) {
         const TileCoord c = tile_coord<BN>(g, t);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, wl)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         const uint32_t idesc = c.bn == BN ? C::kIdesc : idesc_bf16(C::kBMT, c.bn, A_MN, B_MN);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort_flag, wl)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
@@ -745,6 +794,42 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     const int ep_tid = threadIdx.x - 64;     // 0 .. 32*EW - 1
     const int half = (warp - 2) / 4;         // which of the quarter's warps: column blocks half, half + H, ...
     uint8_t* my_stage = epi_stage + (warp - 2) * kEpiWarpBytes;
+    if (TRANS && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL &&
+        (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr)) && blockIdx.x < g.tiles) {
+      // cluster split-K: the aux values (M or the residual) around the rows this
+      // CTA will reduce come into shared memory while the main loop runs.  In
+      // memory a column n of the transposed output holds its rows m
+      // contiguously, so each thread copies whole 16-byte runs of 8 rows (the
+      // rows [ra, rb) are the reduction rows widened to multiples of 8), all
+      // of its loads in flight at once.
+      const TileCoord c = tile_coord<BN>(g, blockIdx.x);
+      const int R = (BM + g.splits - 1) / g.splits;
+      const int r0 = c.split * R, r1 = min(BM, r0 + R);
+      const int ra = r0 & ~7, rb = min(BM, (r1 + 7) & ~7), nr8 = max(0, rb - ra) / 8;
+      const int ncols = min(c.bn, g.N - c.n0);
+      const int chunks = ncols * nr8;
+      bf16* pre = reinterpret_cast<bf16*>(epi_area);
+      const bf16* aux = reinterpret_cast<const bf16*>(g.aux);
+      constexpr int kPre = 8;
+      for (int c0i = ep_tid; c0i < chunks; c0i += kPre * (32 * EW)) {
+        uint4 v[kPre];
+#pragma unroll
+        for (int u = 0; u < kPre; ++u) {
+          const int ch = c0i + u * 32 * EW;
+          const int n = ch < chunks ? ch / nr8 : 0, r8 = ch < chunks ? ch % nr8 : 0;
+          const int m = c.m * BM + ra + 8 * r8;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (ch < chunks && m + 8 <= g.M)   // M is a multiple of 8: runs are whole or outside
+            v[u] = *reinterpret_cast<const uint4*>(aux + static_cast<long long>(c.n0 + n) * g.ldo + m);
+        }
+#pragma unroll
+        for (int u = 0; u < kPre; ++u) {
+          const int ch = c0i + u * 32 * EW;
+          if (ch < chunks)
+            *reinterpret_cast<uint4*>(pre + (ch / nr8) * C::kAuxPitch + 8 * (ch % nr8)) = v[u];
+        }
+      }
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t aux_phase = 0;    // parity bit per aux slot
@@ -773,7 +858,11 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
           for (int i = ep_tid; i < c.bn; i += EPI_THREADS)
             epi_vec[i] = c.n0 + i < g.N ? g.vec[c.n0 + i] : 0.0f;
       }
-      bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag);
+      bool ok = true;
+      // stall_test: auxf[3] is never armed in the element-wise (TRANS) epilogue,
+      // so this wait can only end by running out of its limit
+      if (g.stall_test) ok = mbar_wait(&auxf[3], 0, abort_flag, wl);
+      ok = ok && mbar_wait(&tfull[acc], acc_phase, abort_flag, wl);
       // the split-K and TMA paths synchronise the epilogue warps, so they must
       // agree on leaving the loop together (the barrier also publishes epi_vec)
       if (split || tma) ok = epi_agree<EPI_THREADS>(ok);
@@ -825,7 +914,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
             const int n0 = c.n0 + 64 * j;
             const bool mine = j < C::kSlots && 64 * j < c.bn && n0 < g.N;
             if (has_aux) {
-              ok = mine ? mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag) : true;
+              ok = mine ? mbar_wait(&auxf[j], (aux_phase >> j) & 1u, abort_flag, wl) : true;
               ok = epi_agree<EPI_THREADS>(ok);
               if (!ok) break;
               if (mine) aux_phase ^= 1u << j;
@@ -1005,45 +1094,62 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     const int total = nrows * ((ncols + 3) / 4);
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     const uint32_t base = smem_u32(smem);
-    // kRed elements per thread and pass, every load of a pass issued first
-    constexpr int kRed = 4;
+    const bf16* pre = reinterpret_cast<const bf16*>(epi_area);   // aux rows (TRANS)
+    // kRed elements per thread and pass; every split's loads of a pass are
+    // issued before the first add, and the adds run in split order
+    constexpr int kRed = 2;
+    constexpr int kMaxCsplit = 8;
+    const int ra = r0 & ~7;   // first row of the prefetched aux runs (TRANS)
     for (int e0 = threadIdx.x; e0 < total; e0 += kRed * blockDim.x) {
-      int mm[kRed], nn[kRed];
+      int mm[kRed], nn[kRed], lrs[kRed], lcs[kRed];
       uint32_t off[kRed];
       bool live[kRed];
-      float4 v[kRed];
       float a[kRed][4];
 #pragma unroll
       for (int u = 0; u < kRed; ++u) {
         const int e = e0 + u * static_cast<int>(blockDim.x);
-        const int lr = r0 + (e < total ? e % nrows : 0);
-        const int lc = 4 * (e < total ? e / nrows : 0);
+        lrs[u] = e < total ? e % nrows : 0;
+        lcs[u] = 4 * (e < total ? e / nrows : 0);
+        const int lr = r0 + lrs[u];
         mm[u] = c.m * BM + lr;
-        nn[u] = c.n0 + lc;
+        nn[u] = c.n0 + lcs[u];
         live[u] = e < total && mm[u] < g.M;
-        off[u] = static_cast<uint32_t>(lr * C::kCsplitPitch + lc) * 4u;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const long long o = TRANS ? static_cast<long long>(nn[u] + k) * g.ldo + mm[u]
-                                    : static_cast<long long>(mm[u]) * g.ldo + nn[u] + k;
-          a[u][k] = has_aux && live[u] && nn[u] + k < g.N ? to_f32(reinterpret_cast<const bf16*>(g.aux)[o]) : 0.0f;
-        }
-        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        off[u] = static_cast<uint32_t>(lr * C::kCsplitPitch + lcs[u]) * 4u;
       }
-      for (int sp = 0; sp < g.splits; ++sp) {
-        const uint32_t peer = mapa_shared(base, static_cast<uint32_t>(sp));
-        float4 x[kRed];
+      float4 x[kMaxCsplit][kRed];
 #pragma unroll
-        for (int u = 0; u < kRed; ++u) x[u] = ld_dsmem_f32x4(peer + off[u]);
+      for (int sp = 0; sp < kMaxCsplit; ++sp) {
+        if (sp < g.splits) {
+          const uint32_t peer = mapa_shared(base, static_cast<uint32_t>(sp));
 #pragma unroll
-        for (int u = 0; u < kRed; ++u) {
-          v[u].x += x[u].x; v[u].y += x[u].y; v[u].z += x[u].z; v[u].w += x[u].w;
+          for (int u = 0; u < kRed; ++u) x[sp][u] = ld_dsmem_f32x4(peer + off[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kRed; ++u) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) a[u][k] = 0.0f;
+        if (has_aux && live[u]) {
+          if (TRANS) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              a[u][k] = __bfloat162float(pre[(lcs[u] + k) * C::kAuxPitch + r0 + lrs[u] - ra]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (nn[u] + k < g.N)
+                a[u][k] = to_f32(reinterpret_cast<const bf16*>(g.aux)[static_cast<long long>(mm[u]) * g.ldo + nn[u] + k]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRed; ++u) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int sp = 0; sp < kMaxCsplit; ++sp)
+          if (sp < g.splits) { v.x += x[sp][u].x; v.y += x[sp][u].y; v.z += x[sp][u].z; v.w += x[sp][u].w; }
         if (!live[u]) continue;
-        const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        const float w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (nn[u] + k >= g.N) break;

@@ -133,3 +133,30 @@ class GMULayer:
         ws = self._workspace(("step", rows), abi.gmu_step_workspace(d, rows))
         abi.gmu_step(d, rows, X, M, self.W1, self.W2, X if residual else None, Y, ws, stream)
         return Y
+
+
+class DecodeChain:
+    """One decode token through the scan and a stack of GMU layers that reuse
+    its readout: m_t = scan step(u_t); X <- X + GMU_l(X, m_t) for each layer,
+    as one sambay_decode_step call (states and X updated in place)."""
+
+    def __init__(self, scan: ScanLayer, gmus):
+        self.scan = scan
+        self.gmus = list(gmus)
+        self.layers = abi.make_gmu_layers([(g.W1, g.W2) for g in self.gmus])
+        self._ws = {}
+
+    def step(self, u_t, ssm_state, conv_state, X, m_t=None, stream=None):
+        B = u_t.shape[0]
+        if m_t is None:
+            m_t = torch.empty_like(u_t)
+        d = self.scan.dims(B, 1)
+        n = len(self.gmus)
+        ws = self._ws.get(B)
+        need = abi.sambay_decode_step_workspace(d, n)
+        if ws is None or ws.numel() < need:
+            ws = workspace(need, self.scan.device)
+            self._ws[B] = ws
+        abi.sambay_decode_step(self.scan.abi_w, d, u_t, m_t, ssm_state, conv_state, self.layers, n,
+                               X if n else None, ws, stream)
+        return m_t

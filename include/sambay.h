@@ -140,7 +140,16 @@ SAMBAY_API sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const
 /*
  * sambay_scan_step - one decode token per sequence: the prefill with L = 1
  * on the carried state, updating ssm_state and conv_state IN PLACE [GMU]
- * (constant-size state), [MAMBA].  dims->seqlen is ignored.
+ * (constant-size state), [MAMBA].  dims->seqlen is ignored.  In SAMBAY_BF16
+ * mode this is three kernels over channel slices (about one slice of up to
+ * 48 channels per SM): conv + the slice's partial x_proj sums; their sum in a
+ * fixed slice order; dt_proj + the state update, whose state and weight
+ * slices are copied before it waits for the other two.  ws holds the conv
+ * output, the partial sums, delta and B | C:
+ *   B * (4 Di + 4 ceil(Di / chan) (R + 2N) + 4 R16 + 8 N) bytes (R16 = R
+ *   rounded up to 16), about 7.7 MB for 64 sequences at d_inner 5120.
+ * SAMBAY_F32 runs a chain of float32 kernels that exchange their
+ * intermediates through ws.
  *
  *   u_t [B, Di] io in;  m_t [B, Di] io out (must not alias u_t);
  *   ssm_state [B, Di, N] f32 in/out;  conv_state [B, Di, K] io in/out.
@@ -179,6 +188,55 @@ SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const v
                        const void* W1, const void* W2, const void* residual, void* Y,
                        void* ws, size_t ws_bytes, sambay_stream_t stream);
 
+/* Weights of one Gated Memory Unit layer (device pointers, [Di, Dm] io each). */
+typedef struct {
+  const void* W1; /* used as W1^T: X W1^T maps Dm -> Di   */
+  const void* W2; /* multiplies on the right: Di -> Dm    */
+} sambay_gmu_weights;
+
+/*
+ * sambay_decode_step - one decode token of every sequence through the shared
+ * memory and the cross-decoder layers that reuse it [GMU], [FRAME]:
+ *     m_t = sambay_scan_step(u_t)                    (states updated in place)
+ *     for l in 0 .. n_layers-1:  X <- X + GMU_l(X, m_t)   (in place)
+ * i.e. sambay_scan_step followed by n_layers gmu_step calls with
+ * residual == Y == X, issued as one chain of kernels: each kernel after the
+ * first starts while its predecessor finishes (programmatic dependent launch)
+ * and loads its weights before waiting for it; layer 0's gate GEMM, whose
+ * inputs (X, W1) the scan step does not write, runs its whole main loop before
+ * waiting and only its epilogue (which reads m_t) waits.  Results are the
+ * same bits as the separate calls.
+ *
+ *   u_t [B, Di] io in;  m_t [B, Di] io out;  ssm_state, conv_state in/out as in
+ *   sambay_scan_step;  layers: HOST array of n_layers weight pairs;
+ *   X [B, Dm] io in/out (not used when n_layers == 0; must not alias u_t, m_t);
+ *   ws, ws_bytes: >= sambay_decode_step_workspace(dims, n_layers).
+ * B <= 256.  dims->seqlen is ignored; dims->d_model is the GMU width.
+ */
+SAMBAY_API size_t sambay_decode_step_workspace(const sambay_dims* dims, int32_t n_layers);
+SAMBAY_API sambay_status sambay_decode_step(const sambay_scan_weights* w, const sambay_dims* dims,
+                                            const void* u_t, void* m_t, float* ssm_state,
+                                            void* conv_state, int32_t n_layers,
+                                            const sambay_gmu_weights* layers, void* X, void* ws,
+                                            size_t ws_bytes, sambay_stream_t stream);
+
+/*
+ * sambay_gmu_step_stall_test - a test of the fault detector; the paper has no
+ * counterpart.  Runs gmu_step (bf16 only) with one change: before its first
+ * accumulator, each tensor-core kernel's epilogue waits on a barrier that
+ * nothing arrives at, with every bounded wait limited to wait_limit_cycles
+ * (1 .. 2^32) clock cycles.  That wait therefore runs out: the kernels record
+ * SAMBAY_ERR_TIMEOUT in the device status word, stop their loads and MMAs,
+ * drain what is in flight (itself bounded), free their tensor memory and
+ * return.  Y is unspecified afterwards; sambay_device_status reports the
+ * timeout, and the device stays usable.  Nothing faults, traps or hangs.
+ */
+SAMBAY_API sambay_status sambay_gmu_step_stall_test(const sambay_dims* dims, int64_t rows, const void* X,
+                                                    const void* M, const void* W1, const void* W2,
+                                                    const void* residual, void* Y, void* ws,
+                                                    size_t ws_bytes, uint64_t wait_limit_cycles,
+                                                    sambay_stream_t stream);
+
 /*
  * sambay_scan_step_noalloc - sambay_scan_step for callers that cannot
  * allocate device memory.  The paper has no counterpart; this is a property
@@ -193,12 +251,18 @@ SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const v
  * the library (SAMBAY_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that
  * loads the library until the process exits).  It allocates nothing.
  *
- *   - Sizes whose sambay_scan_step_workspace(dims) exceeds
+ *   - The scratch it needs is what sambay_scan_step_workspace(dims) reports
+ *     (see sambay_scan_step): about 7.7 MB for 64 bf16 sequences at d_inner
+ *     5120, and for SAMBAY_F32 about B * (2 * Di + R + 2N + 64) * 4 bytes.
+ *     Sizes whose sambay_scan_step_workspace(dims) exceeds
  *     SAMBAY_NOALLOC_SCRATCH_BYTES are rejected with SAMBAY_ERR_UNSUPPORTED
- *     before any launch (8 MiB covers 64 sequences at d_inner 5120).
+ *     before any launch; check that query against the limit before relying
+ *     on this entry point for a size.
  *   - The first call on each device looks up the array's device address on
  *     that device (so that device must be current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached per device and not
+ *     looked up again, so it is stale after cudaDeviceReset: do not use this
+ *     entry point across a reset in one process.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; nothing in it needs to start at zero.  Calls that overlap on
  *     the GPU (different streams, or host threads without ordering) race on

@@ -40,6 +40,51 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), f"libsambay does not export {name}"
 
 
+def test_noalloc_limit_matches_the_header():
+    src = open(os.path.join(ROOT, "include", "sambay.h")).read()
+    m = re.search(r"#define\s+SAMBAY_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert m, "SAMBAY_NOALLOC_SCRATCH_BYTES not found in include/sambay.h"
+    assert abi.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_decode_step_argument_errors(lib):
+    d = abi.make_dims(4, 1, 128, 256, 16, 4, 16, abi.BF16)
+    p = _FakePtr(0x10000)
+    layers = abi.make_gmu_layers([(p, p)])
+    # m_t aliases u_t
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_decode_step(_weights(), d, p, p, _FakePtr(0x20000), _FakePtr(0x30000), layers, 1,
+                               _FakePtr(0x40000), p, 0)
+    assert e.value.code == 1
+    # X aliases m_t
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_decode_step(_weights(), d, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                               layers, 1, _FakePtr(0x20000), p, 0)
+    assert e.value.code == 1
+    # a NULL layer weight
+    bad = abi.make_gmu_layers([(p, p)])
+    bad[0].W2 = None
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_decode_step(_weights(), d, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                               bad, 1, _FakePtr(0x50000), p, 0)
+    assert e.value.code == 1
+    # more than 256 sequences
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_decode_step(_weights(), abi.make_dims(300, 1, 128, 256, 16, 4, 16, abi.BF16), p,
+                               _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000), layers, 1,
+                               _FakePtr(0x50000), p, 0)
+    assert e.value.code == 2
+    # workspace too small for the layers' H (1 byte)
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_decode_step(_weights(), d, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                               layers, 1, _FakePtr(0x50000), p, 0)
+    assert e.value.code == 3
+    # the fault-detector test entry point validates like gmu_step
+    with pytest.raises(abi.SambayError) as e:
+        abi.sambay_gmu_step_stall_test(d, 4, p, p, p, p, None, p, p, 0, 0)
+    assert e.value.code == 1
+
+
 def test_status_strings_and_version(lib):
     assert abi.sambay_version() == "0.1.0"
     assert abi.sambay_status_string(0) == "ok"
@@ -63,9 +108,19 @@ def test_workspace_queries(lib):
     want = (r256(T * Di * 4) + r256(9 * T * ldx * 4) + r256(T * ldx * 4) + r256(T * 2 * Rp * 2)
             + r256(T * Di * 4) + r256(T // 2 * 64 * 4))
     assert abi.sambay_scan_prefill_workspace(d) == want
-    assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == \
-        r256(64 * Di * 4) + r256(54 * 64 * ldx * 4) + r256(64 * ldx * 4) + r256(64 * 2 * Rp * 2) \
-        + r256(64 * Di * 4) + r256(64 * 64 * 4)
+    # bf16 decode step: conv output, x_proj partials of 128 slices of 40
+    # channels, the split delta, B | C
+    step64 = r256(64 * Di * 4) + r256(128 * ldx * 64 * 4) + r256(2 * 64 * 160 * 2) + r256(64 * 32 * 4)
+    assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == step64
+    assert step64 <= abi.NOALLOC_SCRATCH_BYTES
+    # float32 decode step: conv output, x_proj output, dt and B | C pairs
+    f64 = abi.make_dims(64, 999, 64, 128, 16, 4, 8, abi.F32)
+    assert abi.sambay_scan_step_workspace(f64) == r256(64 * 128 * 4) + r256(64 * 40 * 4) \
+        + r256(64 * 128 * 4) + r256(64 * 64 * 4)
+    # decode step with GMU layers: the scan step's scratch, then H [B, Di]
+    assert abi.sambay_decode_step_workspace(abi.make_dims(64, 1, 2560, 5120), 8) == step64 + r256(64 * 5120 * 2)
+    assert abi.sambay_decode_step_workspace(abi.make_dims(64, 1, 2560, 5120), 0) == step64
+    assert abi.sambay_decode_step_workspace(abi.make_dims(257, 1, 2560, 5120), 1) == 0
     # float32 mode: no partials, no split delta
     f = abi.make_dims(1, 64, 64, 128, 16, 4, 4, abi.F32)
     assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4) \
@@ -143,8 +198,9 @@ def test_scan_argument_errors(lib):
     with pytest.raises(abi.SambayError) as e:
         abi.sambay_scan_prefill(_weights(), d, p, _FakePtr(0x20000), p, p, True, p, st)
     assert e.value.code == 3
+    d32 = abi.make_dims(1, 16, 64, 128, 16, 4, 8, abi.F32)
     with pytest.raises(abi.SambayError) as e:
-        abi.sambay_scan_step(_weights(), d, p, _FakePtr(0x20000), p, p, p, st)
+        abi.sambay_scan_step(_weights(), d32, p, _FakePtr(0x20000), p, p, p, st)
     assert e.value.code == 3
     with pytest.raises(abi.SambayError) as e:
         abi.sambay_scan_step(_weights(), d, p, p, p, p, p, st)

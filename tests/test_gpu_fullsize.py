@@ -14,7 +14,7 @@ import torch
 from gated_memory_sharing_b200 import abi, synth
 from gated_memory_sharing_b200.layers import GMULayer, ScanLayer, to_device
 from oracle import sambay_ref as ref
-from tests.gpu_util import TOL_BF16, assert_close, host
+from tests.gpu_util import TOL_BF16, assert_close, assert_close_chain, assert_layers_per_layer, host
 
 pytestmark = pytest.mark.gpu
 
@@ -106,7 +106,11 @@ def test_sharing_slice_prefill_b2_l8192_eight_layers():
     rows = np.concatenate([toks, d.seqlen + toks])               # both sequences
     Mrows = np.concatenate([r0[0, toks], r0[1, toks]])
     Xr = ref.gmu_layers_ref(X[rows], Mrows, W1s, W2s)
-    assert_close(host(Xd)[rows], Xr, TOL_BF16, "8-layer sharing chain (sampled rows)")
+    assert_close_chain(host(Xd)[rows], Xr, len(W1s), "8-layer sharing chain (sampled rows)")
+    # every layer on its own at full size, on the oracle's chain state
+    gmus = [GMULayer(W1s[l], W2s[l], abi.BF16) for l in range(len(W1s))]
+    assert_layers_per_layer(lambda l, x, m: gmus[l].forward(x, m, residual=True), to_device(X, abi.BF16), Mflat,
+                            rows, X[rows], Mrows, W1s, W2s, "8-layer sharing chain")
 
 
 def test_sharing_slice_decode_b16_eight_layers():
@@ -127,5 +131,8 @@ def test_sharing_slice_decode_b16_eight_layers():
         x = to_device(X0[i], abi.BF16)
         for g in gmus:
             g.step(x, m, residual=True, Y=x)
-        xr = ref.gmu_layers_ref(X0[i], r["M"][:, L0 + i], [g["W1"] for g in gws], [g["W2"] for g in gws])
-        assert_close(host(x), xr, TOL_BF16, f"decode step {i}: 8-layer chain")
+        W1s, W2s = [g["W1"] for g in gws], [g["W2"] for g in gws]
+        xr = ref.gmu_layers_ref(X0[i], r["M"][:, L0 + i], W1s, W2s)
+        assert_close_chain(host(x), xr, len(gws), f"decode step {i}: 8-layer chain")
+        assert_layers_per_layer(lambda l, xx, mm: gmus[l].step(xx, mm, residual=True), to_device(X0[i], abi.BF16), m,
+                                np.arange(B), X0[i], r["M"][:, L0 + i], W1s, W2s, f"decode step {i}")

@@ -63,7 +63,7 @@ def _ref_worker(rank, world, port, out):
     import bench
 
     class A:
-        steps, warmup, gpus = 1, 0, world
+        steps, warmup, gpus, workload = 1, 0, world, bench.HEADLINE
     buf = io.StringIO()
     orig = bench.synth.workload
     bench.synth.workload = lambda name: orig("tiny_f32")      # a small stand-in
