@@ -301,7 +301,7 @@ def lifted_gmu_ref(uc, G, mix, W2):
 # the GMU in the cross-decoder
 # --------------------------------------------------------------------------
 
-def mamba_layer_ref(X, w, W_in, W_z, W_out, ssm_state=None, conv_state=None, residual=True):
+def mamba_layer_ref(X, w, W_in, W_z, W_out, ssm_state=None, conv_state=None, residual=True, io_round=False):
     """The whole Mamba layer whose scan readout is the shared memory M.
 
     Mamba block (Gu & Dao 2023, section 3.4): the input is projected into two
@@ -315,12 +315,20 @@ def mamba_layer_ref(X, w, W_in, W_z, W_out, ssm_state=None, conv_state=None, res
     transposed); W_out [Di, Dm], multiplying on the right (out_proj's weight
     transposed).  Returns dict(out [B, L, Dm] (+X when ``residual``), M = y,
     z, u, ssm_state, conv_state).
+
+    ``io_round``: the layer's steps exchange u (projection -> scan) and M
+    (scan -> gated output projection) as bfloat16 tensors, the I/O type of the
+    bf16 workloads; the scan then runs on the bf16 rounding of the exact u,
+    and the output projection reads the bf16 rounding of the exact M.  The
+    arithmetic inside each step stays float64.
     """
     X = _f64(X)
     u = X @ _f64(W_in).T
     z = X @ _f64(W_z).T
+    if io_round:
+        u = round_bf16(u)
     r = scan_prefill_ref(u, w, ssm_state, conv_state)
-    out = (r["M"] * silu(z)) @ _f64(W_out)
+    out = ((round_bf16(r["M"]) if io_round else r["M"]) * silu(z)) @ _f64(W_out)
     if residual:
         out = out + X
     return dict(out=out, M=r["M"], z=z, u=u, ssm_state=r["ssm_state"], conv_state=r["conv_state"])

@@ -92,6 +92,24 @@ def test_mamba_layer_matches_torch_linear_composition():
     np.testing.assert_allclose(r["M"], y, rtol=1e-13)
 
 
+def test_mamba_layer_io_round_rounds_u_and_M():
+    rng = np.random.default_rng(8)
+    B, L, Dm, Di = 1, 11, 5, 6
+    w = _scan_weights(rng, Di)
+    X = rng.standard_normal((B, L, Dm))
+    W_in, W_z, W_out = (rng.standard_normal((Di, Dm)) * 0.5 for _ in range(3))
+    r = ref.mamba_layer_ref(X, w, W_in, W_z, W_out, io_round=True)
+    bf = lambda t: t.to(torch.bfloat16).to(torch.float64)
+    Xt = torch.from_numpy(X)
+    u = bf(F.linear(Xt, torch.from_numpy(W_in)))
+    z = F.linear(Xt, torch.from_numpy(W_z))
+    y = ref.scan_prefill_ref(u.numpy(), w)["M"]
+    out = F.linear(bf(torch.from_numpy(y)) * F.silu(z), torch.from_numpy(W_out).T) + Xt
+    np.testing.assert_allclose(r["M"], y, rtol=1e-13)
+    np.testing.assert_allclose(r["out"], out.numpy(), rtol=1e-12, atol=1e-13)
+    assert not np.allclose(r["M"], ref.mamba_layer_ref(X, w, W_in, W_z, W_out)["M"], rtol=1e-6)
+
+
 def test_mamba_layer_special_cases():
     rng = np.random.default_rng(3)
     B, L, Di = 1, 7, 6
