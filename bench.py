@@ -15,6 +15,11 @@ method are measured in the same run and reported under "workloads":
                            layers (X <- X + GMU_l(X, M))
   sharing_decode_b16       16 sequences decoding through the scan step and
                            the 8 GMU layers
+  cross_attn_vs_gmu_b64    one decoded token of 64 sequences through a
+                           cross-attention layer over the KV cache (2048 and
+                           34816 cached tokens: the 2K prompt and the end of
+                           32K generated ones) and through a GMU layer: bytes
+                           and time per decoded token of each
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--only-headline] [--no-cpu-baseline]
@@ -44,7 +49,7 @@ from gated_memory_sharing_b200 import synth  # noqa: E402
 
 HEADLINE = "prefill_b1_l2048"
 WORKLOADS = ("prefill_b1_l2048", "decode_b64", "long_prefill_b4_l32768", "sharing_b2_l8192",
-             "sharing_decode_b16")
+             "sharing_decode_b16", "cross_attn_vs_gmu_b64")
 UNIT = "tokens/s"
 METRICS = {
     "prefill_b1_l2048": "scan+GMU prefill tokens/s",
@@ -52,6 +57,7 @@ METRICS = {
     "long_prefill_b4_l32768": "scan+GMU prefill tokens/s",
     "sharing_b2_l8192": "scan+8xGMU prefill tokens/s",
     "sharing_decode_b16": "scan+8xGMU decode tokens/s",
+    "cross_attn_vs_gmu_b64": "cross-attention decode tokens/s at 2048 cached tokens",
 }
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from an
 # earlier ncu capture of the headline workload, for kernels unchanged since
@@ -207,7 +213,10 @@ def dev_normal(shape, seed, device):
 
 
 def workload_dims(name):
-    """(dims, seed, gmu layers, decode batch or None, decode prompt) of a bench workload."""
+    """(dims, seed, gmu layers, decode?) of a bench workload."""
+    if name == "cross_attn_vs_gmu_b64":
+        d, seed = synth.workload("decode_b64")
+        return d, seed, 1, False
     if name == "sharing_decode_b16":
         d, seed = synth.workload("sharing_b2_l8192")
         return (synth.Dims(synth.SHARING_DECODE_BATCH, 1024, d.d_model, d.d_inner, d.d_state, d.d_conv,
@@ -248,9 +257,20 @@ def cpu_baseline(name, budget_s=8.0, reps_max=4):
     sequence; decode steps of every sequence of the batch."""
     from oracle import sambay_ref as ref
     d, seed, layers, decode = workload_dims(name)
+    cores = len(os.sched_getaffinity(0))
+    if name == "cross_attn_vs_gmu_b64":
+        S, N = 4, d.seqlen
+        q, K, V = synth.attention_inputs(S, N, synth.ATTN_Q_HEADS, synth.ATTN_KV_HEADS, synth.ATTN_HEAD_DIM, seed)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 20 and (reps == 0 or time.perf_counter() - t0 < budget_s):
+            ref.cross_attention_decode_ref(q, K, V)
+            reps += 1
+        el = time.perf_counter() - t0
+        return {"value": reps * S / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"cross-attention decode of {S} sequences over {N} cached tokens x {reps}, "
+                          f"{el:.1f} s of float64 NumPy"}
     w = synth.scan_weights(d, seed)
     gws = [synth.gmu_weights(d, seed, layer=l) for l in range(layers)]
-    cores = len(os.sched_getaffinity(0))
     if decode:
         B = d.batch
         dd = synth.Dims(B, 16, d.d_model, d.d_inner, d.d_state, d.d_conv, d.dt_rank, synth.BF16)
@@ -628,6 +648,84 @@ def bench_decode(args, ctx, name):
     }
 
 
+# --------------------------------------------------------------------- our arm: attention vs GMU
+
+def bench_attn_vs_gmu(args, ctx, name):
+    """The pages' decode I/O claim on this machine: a cross-attention layer reads
+    the whole KV cache per decoded token, a GMU layer its two weight matrices
+    (shared by the batch)."""
+    import torch
+    from gated_memory_sharing_b200 import abi
+    from gated_memory_sharing_b200.layers import GMULayer, workspace
+    world, rank, device, flush, stream, peaks, peak_kind, sms = ctx
+    d, seed = synth.workload("decode_b64")
+    B, Dm, Di = d.batch, d.d_model, d.d_inner
+    Hq, Hkv, dh = synth.ATTN_Q_HEADS, synth.ATTN_KV_HEADS, synth.ATTN_HEAD_DIM
+    rs = seed + 7919 * rank
+    res = {}
+    steps = max(5, min(args.steps, 20))
+
+    def timed(fn):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for _ in range(3):
+            fn()
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush(i)
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device) / steps
+
+    n_max = synth.DECODE_STEPS["decode_b64"] + d.seqlen
+    q = dev_normal((B, Hq, dh), rs, device)
+    Kc = dev_normal((B, n_max, Hkv, dh), rs + 1, device)
+    Vc = dev_normal((B, n_max, Hkv, dh), rs + 2, device)
+    out = torch.empty(B, Hq, dh, dtype=torch.bfloat16, device=device)
+    for N in (d.seqlen, n_max):
+        # the first N tokens of each sequence's cache: [B, N, Hkv, dh] views of the
+        # full cache are not dense, so each length has its own dense copy
+        K = Kc[:, :N].contiguous()
+        V = Vc[:, :N].contiguous()
+        dims = abi.AttnDims(B, N, Hq, Hkv, dh)
+        ws = workspace(abi.sambay_cross_attn_decode_workspace(dims), device)
+        ms = timed(lambda: abi.sambay_cross_attn_decode(dims, q, K, V, out, 0.0, ws))
+        nbytes = 2 * B * N * Hkv * dh * 2 + 2 * B * Hq * dh * 2
+        res[N] = {"cached_tokens": N, "us_per_step": 1e3 * ms, "bytes_per_step": nbytes,
+                  "bytes_per_decoded_token": nbytes / B, "tokens_per_s": world * B / (ms / 1e3),
+                  "achieved_gbs": nbytes / (ms / 1e3) / 1e9}
+        del K, V
+    del Kc, Vc
+    gw = synth.gmu_weights(d, seed)
+    gmu = GMULayer(gw["W1"], gw["W2"], abi.BF16)
+    X = dev_normal((B, Dm), rs + 3, device)
+    M = dev_normal((B, Di), rs + 4, device)
+    Y = torch.empty_like(X)
+    ms_g = timed(lambda: gmu.step(X, M, residual=True, Y=Y))
+    gbytes = 2 * Di * Dm * 2 + B * (2 * Dm + Di + Dm) * 2
+    a0 = res[d.seqlen]
+    return {
+        "metric": METRICS[name], "value": a0["tokens_per_s"], "unit": UNIT, "ms_per_step": a0["us_per_step"] / 1e3,
+        "steps": steps,
+        "config": {"workload": name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": dh, "d_model": Dm,
+                   "d_inner": Di, "cached_tokens": [d.seqlen, n_max]},
+        "l2": "flushed before every timed call (256 MB write + 256 MB read, outside the events)",
+        "cross_attention": list(res.values()),
+        "gmu_layer": {"us_per_step": 1e3 * ms_g, "bytes_per_step": gbytes, "bytes_per_decoded_token": gbytes / B,
+                      "tokens_per_s": world * B / (ms_g / 1e3), "achieved_gbs": gbytes / (ms_g / 1e3) / 1e9},
+        "bytes_per_token_ratio": {str(N): r["bytes_per_decoded_token"] / (gbytes / B) for N, r in res.items()},
+        "time_ratio": {str(N): r["us_per_step"] / (1e3 * ms_g) for N, r in res.items()},
+        "roofline": {"bound": "hbm", "achieved": a0["achieved_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": a0["achieved_gbs"] / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "cross_attn_decode (2048 cached tokens)", "peak_note": f"{peak_kind} HBM copy"},
+        "e2e": None,
+        "gpu_launches": steps,
+    }
+
+
 def run_ours(args, world, rank, local):
     import torch
     from gated_memory_sharing_b200 import abi, build
@@ -650,6 +748,9 @@ def run_ours(args, world, rank, local):
     time.sleep(0.3)
     results = {}
     for name in names:
+        if name == "cross_attn_vs_gmu_b64":
+            results[name] = bench_attn_vs_gmu(args, ctx, name)
+            continue
         fn = bench_decode if workload_dims(name)[3] else bench_prefill
         results[name] = fn(args, ctx, name)
         torch.cuda.synchronize()

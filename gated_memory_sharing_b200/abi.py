@@ -38,8 +38,14 @@ EXPORTS = (
     "sambay_scan_step_noalloc",
     "gmu_forward",
     "gmu_step",
+    "sambay_in_proj_workspace",
+    "sambay_in_proj",
+    "sambay_mlp_memory_workspace",
+    "sambay_mlp_memory",
     "sambay_decode_step_workspace",
     "sambay_decode_step",
+    "sambay_cross_attn_decode_workspace",
+    "sambay_cross_attn_decode",
     "sambay_gmu_step_stall_test",
     "sambay_profile_begin",
     "sambay_profile_end",
@@ -80,6 +86,16 @@ class ScanWeights(ctypes.Structure):
     ]
 
 
+class AttnDims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("kv_len", ctypes.c_int32),
+        ("q_heads", ctypes.c_int32),
+        ("kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+    ]
+
+
 class GmuWeights(ctypes.Structure):
     _fields_ = [
         ("W1", ctypes.c_void_p),
@@ -103,6 +119,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
     pd, pw = ctypes.POINTER(Dims), ctypes.POINTER(ScanWeights)
     pg = ctypes.POINTER(GmuWeights)
+    pa = ctypes.POINTER(AttnDims)
     sig = {
         "sambay_scan_prefill_workspace": (sz, [pd]),
         "sambay_scan_step_workspace": (sz, [pd]),
@@ -113,7 +130,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sambay_scan_step_noalloc": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp]),
         "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sambay_in_proj_workspace": (sz, [pd, i64]),
+        "sambay_in_proj": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, sz, vp]),
+        "sambay_mlp_memory_workspace": (sz, [pd, i64]),
+        "sambay_mlp_memory": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, sz, vp]),
         "sambay_decode_step_workspace": (sz, [pd, i32]),
+        "sambay_cross_attn_decode_workspace": (sz, [pa]),
+        "sambay_cross_attn_decode": (ctypes.c_int, [pa, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp]),
         "sambay_decode_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, i32, pg, vp, vp, sz, vp]),
         "sambay_gmu_step_stall_test": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz,
                                                       ctypes.c_uint64, vp]),
@@ -190,6 +213,36 @@ def sambay_scan_step(weights: ScanWeights, dims: Dims, u_t, m_t, ssm_state, conv
     _check("sambay_scan_step", load().sambay_scan_step(
         ctypes.byref(weights), ctypes.byref(dims), _p(u_t), _p(m_t), _p(ssm_state),
         _p(conv_state), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_in_proj_workspace(dims: Dims, rows: int) -> int:
+    return load().sambay_in_proj_workspace(ctypes.byref(dims), rows)
+
+
+def sambay_in_proj(dims: Dims, rows: int, X, W_in, u, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_in_proj", load().sambay_in_proj(
+        ctypes.byref(dims), rows, _p(X), _p(W_in), _p(u), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_mlp_memory_workspace(dims: Dims, rows: int) -> int:
+    return load().sambay_mlp_memory_workspace(ctypes.byref(dims), rows)
+
+
+def sambay_mlp_memory(dims: Dims, rows: int, X, W_g, W_u, M, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_mlp_memory", load().sambay_mlp_memory(
+        ctypes.byref(dims), rows, _p(X), _p(W_g), _p(W_u), _p(M), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_cross_attn_decode_workspace(dims: AttnDims) -> int:
+    return load().sambay_cross_attn_decode_workspace(ctypes.byref(dims))
+
+
+def sambay_cross_attn_decode(dims: AttnDims, q, K, V, out, scale: float, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_cross_attn_decode", load().sambay_cross_attn_decode(
+        ctypes.byref(dims), _p(q), _p(K), _p(V), _p(out), scale, _p(ws), ws_bytes, _stream(stream)))
 
 
 def sambay_decode_step_workspace(dims: Dims, n_layers: int) -> int:

@@ -7,12 +7,14 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <vector>
 
 #include "../../include/sambay.h"
 #include "common.cuh"
+#include "attn_kernels.cuh"
 #include "scan_kernels.cuh"
 #include "simt_gemm.cuh"
 #include "step_kernels.cuh"
@@ -901,6 +903,51 @@ sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* 
   return SAMBAY_OK;
 }
 
+// Y [rows, N] = X [rows, K] W^T, W [N, K] (bf16): KIND = EPI_RESID with no aux
+// is the plain projection, KIND = EPI_GATE gives Y = aux ⊙ SiLU(X W^T).  Up to
+// 256 rows it is the swap-AB decode GEMM (W is the A operand and streams once,
+// split-K over a cluster, reduced through distributed shared memory);
+// otherwise the CTA-pair GEMM, whose last round of tiles may be split along K
+// into `tail`.
+template <int KIND>
+sambay_status project_tc(int dev, int sms, long long rows, int N, int K, const void* X, const void* W,
+                         const void* aux, void* Y, float* tail, size_t tail_bytes, const char* name,
+                         const char* tail_name, cudaStream_t st) {
+  if (rows <= kStepMaxRows) {
+    auto g = tc_args(N, static_cast<int>(rows), K, Y, N, aux);
+    g.csplit = 1;
+    const Operand w{W, N, K}, x{X, rows, K};
+    if (rows <= 32) return run_tc<32, false, false, KIND, true>(name, dev, sms, w, x, g, kStepMaxSplits, st, false);
+    if (rows <= 64) return run_tc<64, false, false, KIND, true>(name, dev, sms, w, x, g, kStepMaxSplits, st, false);
+    if (rows <= 128) return run_tc<128, false, false, KIND, true>(name, dev, sms, w, x, g, kStepMaxSplits, st, false);
+    if (rows <= 192) return run_tc<192, false, false, KIND, true>(name, dev, sms, w, x, g, kStepMaxSplits, st, false);
+    return run_tc<256, false, false, KIND, true>(name, dev, sms, w, x, g, kStepMaxSplits, st, false);
+  }
+  return run_tc<256, false, false, KIND, false, 8, true>(name, dev, sms, Operand{X, rows, K}, Operand{W, N, K},
+                                                         tc_args(static_cast<int>(rows), N, K, Y, N, aux), 1, st,
+                                                         false, true, tail, tail_bytes, tail_name);
+}
+
+// Workspace of the projections: the K-split tail's partial tiles (more than
+// 256 rows), after an optional [rows, N] io buffer.
+struct ProjWs {
+  size_t buf, tail, tail_bytes, total;
+};
+
+ProjWs proj_ws_layout(const sambay_dims* d, long long rows, bool buffer) {
+  ProjWs w{};
+  size_t off = 0;
+  w.buf = off;
+  if (buffer) off += round256(static_cast<size_t>(rows) * d->d_inner * io_bytes(d->io));
+  if (d->io == SAMBAY_BF16 && rows > kStepMaxRows) {
+    w.tail = off;
+    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4;
+    off += round256(w.tail_bytes);
+  }
+  w.total = off;
+  return w;
+}
+
 // How a decode GMU layer's kernels chain onto the work before them.
 struct StepChain {
   bool chained = false;      // the gate GEMM follows a kernel of this call (PDL)
@@ -1154,6 +1201,173 @@ sambay_status sambay_gmu_step_stall_test(const sambay_dims* d, int64_t rows, con
   ch.stall_test = 1;
   return gmu_step_tc(dev, sms, d, rows, X, M, W1, W2, residual, Y, static_cast<uint8_t*>(ws) + L.h, ch,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sambay_in_proj_workspace(const sambay_dims* d, int64_t rows) {
+  if (check_dims(d, true, false) != SAMBAY_OK || rows < 1) return 0;
+  return proj_ws_layout(d, rows, false).total;
+}
+
+sambay_status sambay_in_proj(const sambay_dims* d, int64_t rows, const void* X, const void* W_in, void* u,
+                             void* ws, size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, true, false));
+  if (rows < 1 || rows > (1LL << 30)) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({X, W_in, u}));
+  if (u == X) return SAMBAY_ERR_INVALID_ARG;
+  const ProjWs L = proj_ws_layout(d, rows, false);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int Dm = d->d_model, Di = d->d_inner;
+  if (d->io == SAMBAY_F32)
+    return run_simt<sambay::simt::F32_STORE>("in_proj_f32",
+        simt_args(static_cast<const float*>(X), Dm, 1, static_cast<const float*>(W_in), 1, Dm,
+                  static_cast<int>(rows), Di, Dm, static_cast<float*>(u), Di), st);
+  float* tail = L.tail_bytes ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.tail) : nullptr;
+  return project_tc<sambay::tc::EPI_RESID>(dev, sms, rows, Di, Dm, X, W_in, nullptr, u, tail, L.tail_bytes,
+                                           "in_proj", "in_proj_tail", st);
+}
+
+size_t sambay_mlp_memory_workspace(const sambay_dims* d, int64_t rows) {
+  if (check_dims(d, true, false) != SAMBAY_OK || rows < 1) return 0;
+  return proj_ws_layout(d, rows, true).total;
+}
+
+sambay_status sambay_mlp_memory(const sambay_dims* d, int64_t rows, const void* X, const void* W_g,
+                                const void* W_u, void* M, void* ws, size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, true, false));
+  if (rows < 1 || rows > (1LL << 30)) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({X, W_g, W_u, M}));
+  if (M == X) return SAMBAY_ERR_INVALID_ARG;
+  const ProjWs L = proj_ws_layout(d, rows, true);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int Dm = d->d_model, Df = d->d_inner, T = static_cast<int>(rows);
+  if (d->io == SAMBAY_F32) {
+    float* U = reinterpret_cast<float*>(w8 + L.buf);
+    SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("mlp_up_f32",
+        simt_args(static_cast<const float*>(X), Dm, 1, static_cast<const float*>(W_u), 1, Dm, T, Df, Dm, U, Df), st));
+    return run_simt<sambay::simt::GATE>("mlp_gate_f32",
+        simt_args(static_cast<const float*>(X), Dm, 1, static_cast<const float*>(W_g), 1, Dm, T, Df, Dm,
+                  static_cast<float*>(M), Df, U), st);
+  }
+  bf16* U = reinterpret_cast<bf16*>(w8 + L.buf);
+  float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
+  // U = X W_u^T, then M = U ⊙ SiLU(X W_g^T): the gate GEMM with U as its aux
+  SAMBAY_TRY(project_tc<sambay::tc::EPI_RESID>(dev, sms, rows, Df, Dm, X, W_u, nullptr, U, tail, L.tail_bytes,
+                                               "mlp_up", "mlp_up_tail", st));
+  return project_tc<sambay::tc::EPI_GATE>(dev, sms, rows, Df, Dm, X, W_g, U, M, tail, L.tail_bytes, "mlp_gate",
+                                          "mlp_gate_tail", st);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Split-KV plan of the cross-attention decode: enough (sequence, KV head,
+// split) CTAs to cover a 148-SM B200 about three times, splits of whole
+// 128-token blocks (a function of the sizes only).
+struct AttnPlan {
+  int splits = 1, chunk = 0;
+  size_t o_part = 0, ml_part = 0, total = 0;
+};
+
+sambay_status attn_check(const sambay_attn_dims* a) {
+  if (!a) return SAMBAY_ERR_INVALID_ARG;
+  if (a->batch < 1 || a->kv_len < 1 || a->q_heads < 1 || a->kv_heads < 1 || a->head_dim < 1)
+    return SAMBAY_ERR_INVALID_ARG;
+  if (a->head_dim != 64 && a->head_dim != 128) return SAMBAY_ERR_UNSUPPORTED;
+  if (a->q_heads % a->kv_heads != 0 || a->q_heads / a->kv_heads > 16) return SAMBAY_ERR_UNSUPPORTED;
+  return SAMBAY_OK;
+}
+
+AttnPlan attn_plan(const sambay_attn_dims* a) {
+  AttnPlan pl;
+  constexpr int kBlock = sambay::attn::kTile * sambay::attn::kWarps;
+  const long long pairs = static_cast<long long>(a->batch) * a->kv_heads;
+  const long long blocks = (a->kv_len + kBlock - 1) / kBlock;
+  long long splits = std::max(1LL, (3LL * kSplitTarget + pairs - 1) / pairs);
+  splits = std::min(splits, blocks);
+  pl.chunk = static_cast<int>((blocks + splits - 1) / splits) * kBlock;
+  pl.splits = static_cast<int>((a->kv_len + pl.chunk - 1) / pl.chunk);
+  if (pl.splits > 1) {
+    const size_t qh = static_cast<size_t>(a->batch) * a->q_heads * pl.splits;
+    pl.o_part = 0;
+    pl.ml_part = round256(qh * a->head_dim * 4);
+    pl.total = pl.ml_part + round256(qh * 2 * 4);
+  }
+  return pl;
+}
+
+template <int DH>
+sambay_status attn_launch(int dev, int sms, sambay::attn::AttnParams& p, cudaStream_t st) {
+  using namespace sambay::attn;
+  auto kern = cross_attn_decode_kernel<DH>;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnLayout<DH>::kBytes) !=
+        cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  {
+    ProfScope ps("cross_attn_decode", st);
+    if (launch_k(kern, dim3(p.splits, p.Hkv, p.B), dim3(kThreads), AttnLayout<DH>::kBytes, st, false, 1, p) !=
+        cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+  }
+  if (p.splits > 1) {
+    const long long n = static_cast<long long>(p.B) * p.Hq * DH;
+    ProfScope ps("cross_attn_combine", st);
+    if (launch_k(cross_attn_combine_kernel<DH>, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, st,
+                 true, 1, p) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+  }
+  return SAMBAY_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sambay_cross_attn_decode_workspace(const sambay_attn_dims* a) {
+  if (attn_check(a) != SAMBAY_OK) return 0;
+  return attn_plan(a).total;
+}
+
+sambay_status sambay_cross_attn_decode(const sambay_attn_dims* a, const void* q, const void* K, const void* V,
+                                       void* out, float scale, void* ws, size_t ws_bytes,
+                                       sambay_stream_t stream) {
+  SAMBAY_TRY(attn_check(a));
+  SAMBAY_TRY(check_ptrs({q, K, V, out}));
+  if (out == q || out == K || out == V) return SAMBAY_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || scale > 1e4f) return SAMBAY_ERR_INVALID_ARG;   // also rejects NaN
+  const AttnPlan pl = attn_plan(a);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, pl.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  sambay::attn::AttnParams p{};
+  p.q = static_cast<const bf16*>(q);
+  p.K = static_cast<const bf16*>(K);
+  p.V = static_cast<const bf16*>(V);
+  p.out = static_cast<bf16*>(out);
+  p.o_part = pl.splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.o_part) : nullptr;
+  p.ml_part = pl.splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.ml_part) : nullptr;
+  p.B = a->batch;
+  p.N = a->kv_len;
+  p.Hq = a->q_heads;
+  p.Hkv = a->kv_heads;
+  p.G = a->q_heads / a->kv_heads;
+  p.splits = pl.splits;
+  p.chunk = pl.chunk;
+  const float sc = scale > 0.0f ? scale : 1.0f / sqrtf(static_cast<float>(a->head_dim));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return a->head_dim == 64 ? attn_launch<64>(dev, sms, p, st) : attn_launch<128>(dev, sms, p, st);
 }
 
 sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const sambay_dims* d,

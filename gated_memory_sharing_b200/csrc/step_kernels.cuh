@@ -54,6 +54,7 @@ constexpr int kMaxGroup = 64;    // sequences per CTA (MMA N = 128: 16 n-blocks)
 constexpr int kStateN = 16;      // d_state
 constexpr int kConvK = 4;        // d_conv
 constexpr int kRedLanes = 8;     // lanes per output in step_reduce
+constexpr int kMaxPerLane = 19;  // slices per lane (148 slices at most)
 
 struct StepParams {
   const bf16* u_t;        // [B, Di]
@@ -267,11 +268,17 @@ __global__ void __launch_bounds__(kThreads) step_reduce_kernel(const StepParams 
        w * (32 / kRedLanes) < total; w += warps) {
     const long long o = w * (32 / kRedLanes) + lane / kRedLanes;   // = j * B + s
     const bool valid = o < total;
-    float acc = 0.0f;
-    if (valid) {
-#pragma unroll 4
-      for (int sl = sub; sl < p.nslice; sl += kRedLanes) acc += __ldcg(p.part + sl * slice_stride + o);
+    // every load of the lane in flight at once (nslice <= 8 * kMaxPerLane),
+    // then the adds in slice order
+    float x[kMaxPerLane];
+#pragma unroll
+    for (int k = 0; k < kMaxPerLane; ++k) {
+      const int sl = sub + k * kRedLanes;
+      x[k] = (valid && sl < p.nslice) ? __ldcg(p.part + sl * slice_stride + o) : 0.0f;
     }
+    float acc = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kMaxPerLane; ++k) acc += x[k];
 #pragma unroll
     for (int off = kRedLanes / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (!valid || sub != 0) continue;

@@ -128,6 +128,11 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
                : "memory");
   return v;
 }
+__device__ __forceinline__ void st_dsmem_f32x4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
 // TMA load into this CTA's shared memory whose bytes complete on the
 // leader CTA's barrier
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
@@ -503,7 +508,12 @@ struct Cfg {
   static constexpr int kStageArea = TRANS ? BN * kAuxPitch * 2
                                           : (kSlots * kSlotBytes > EW * kEpiWarpBytes ? kSlots * kSlotBytes
                                                                                      : EW * kEpiWarpBytes);
-  static constexpr int kEpiBytes = kStageArea + (kTmaEpi ? 1024 /*bias*/ : 0);
+  // cluster split-K with tiles of at most 64 columns (decode batches up to 64):
+  // the splits push their partial rows into the reducing CTA's receive buffer
+  // ([split][row of the CTA's slice][kCsplitPitch], at most BM + 8 rows)
+  static constexpr bool kPush = TRANS && BN <= 64;
+  static constexpr int kRecvBytes = kPush ? (BM + 8) * (BN + 4) * 4 : 0;
+  static constexpr int kEpiBytes = kStageArea + kRecvBytes + (kTmaEpi ? 1024 /*bias*/ : 0);
   static constexpr int kFixed = 1024 /*align slack*/ + 512 /*barriers*/ + kEpiBytes;
   static constexpr int kStagesFit = (kMaxDynSmem - kFixed) / kStageBytes;
   static constexpr int kStageCap = 8;
@@ -990,8 +1000,21 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             __stcg(reinterpret_cast<float4*>(part + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+        } else if (split && g.csplit && C::kPush) {
+          // cluster split-K, push: tile row r belongs to the CTA (cluster rank)
+          // r / R that reduces it; this split's 32 values of the row go
+          // straight into that CTA's receive buffer (distributed shared
+          // memory stores, no wait), at [split * R + r % R]
+          const int r = quarter * 32 + lane;
+          const int R = (BM + g.splits - 1) / g.splits;
+          const int owner = r / R;
+          const uint32_t local = smem_u32(epi_area + C::kStageArea) +
+                                 static_cast<uint32_t>(((c.split * R + r - owner * R) * C::kCsplitPitch + ch * 32) * 4);
+          const uint32_t remote = mapa_shared(local, static_cast<uint32_t>(owner));
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) st_dsmem_f32x4(remote + 4u * j, make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
         } else if (split && g.csplit) {
-          // cluster split-K: this split's partial tile stays in this CTA's
+          // cluster split-K, pull: this split's partial tile stays in this CTA's
           // (now idle) pipeline shared memory, row-major at kCsplitPitch; the
           // cluster's CTAs read it there after the cluster barrier
           float* dst = reinterpret_cast<float*>(smem) + (quarter * 32 + lane) * C::kCsplitPitch + ch * 32;
@@ -1079,8 +1102,46 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
   if (PAIR) cluster_sync();
   else __syncthreads();
   tc_fence_after();
-  if (!PAIR && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {
-    // cluster split-K: every CTA of the cluster holds its partial tile in its
+  if (!PAIR && C::kPush && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {
+    // cluster split-K, push: every split has stored its rows into the
+    // reducing CTAs' receive buffers; after one cluster barrier (which orders
+    // those stores) each CTA sums its rows [split * R, +R) locally, in split
+    // order, and applies the final op.  Nothing touches a peer's shared
+    // memory after the barrier, so no second barrier is needed before exit.
+    // Thread: 4 consecutive columns of one row, consecutive threads on
+    // consecutive rows.
+    cluster_sync();
+    const TileCoord c = tile_coord<BN>(g, blockIdx.x);
+    const int R = (BM + g.splits - 1) / g.splits;
+    const int r0 = c.split * R, r1 = min(BM, r0 + R);
+    const int nrows = max(0, r1 - r0), ncols = min(c.bn, g.N - c.n0);
+    const int total = nrows * ((ncols + 3) / 4);
+    const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
+    const float* recv = reinterpret_cast<const float*>(epi_area + C::kStageArea);
+    const bf16* pre = reinterpret_cast<const bf16*>(epi_area);
+    const int ra = r0 & ~7;
+    // (compact loops: this code runs once per CTA, so its instructions are
+    // fetched cold; a short body costs less than an unrolled one)
+#pragma unroll 1
+    for (int e = threadIdx.x; e < total; e += blockDim.x) {
+      const int lr = e % nrows, lc = 4 * (e / nrows);
+      const int mm = c.m * BM + r0 + lr, nn = c.n0 + lc;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int sp = 0; sp < g.splits; ++sp) {
+        const float4 x = *reinterpret_cast<const float4*>(recv + (sp * R + lr) * C::kCsplitPitch + lc);
+        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+      }
+      if (mm >= g.M) continue;
+      const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll 1
+      for (int k = 0; k < 4 && nn + k < g.N; ++k) {
+        const float a = has_aux ? __bfloat162float(pre[(lc + k) * C::kAuxPitch + r0 + lr - ra]) : 0.0f;
+        epi_store_one<KIND>(g, static_cast<long long>(nn + k) * g.ldo + mm, nn + k, w[k], a);
+      }
+    }
+  } else if (!PAIR && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {
+    // cluster split-K, pull: every CTA of the cluster holds its partial tile in its
     // shared memory; CTA `split` (cluster rank `split`) sums rows
     // [split * R, +R) of the tile over the splits in split order, reading the
     // peers' tiles 16 bytes at a time through distributed shared memory, and

@@ -160,3 +160,70 @@ class DecodeChain:
         abi.sambay_decode_step(self.scan.abi_w, d, u_t, m_t, ssm_state, conv_state, self.layers, n,
                                X if n else None, ws, stream)
         return m_t
+
+
+class MambaLayer:
+    """The whole Mamba layer whose scan readout is the shared memory M:
+    u = X W_in^T, y = scan(u) (= M), out = (y ⊙ SiLU(X W_z^T)) W_out + X.
+    The gated output projection is the GMU's computation with W1 = W_z and
+    W2 = W_out, so it runs through gmu_forward / gmu_step."""
+
+    def __init__(self, w: dict, bw: dict, d_model: int, io: int, device="cuda"):
+        self.scan = ScanLayer(w, d_model, io, device)
+        self.W_in = to_device(bw["W_in"], io, device)
+        self.gate = GMULayer(bw["W_z"], bw["W_out"], io, device)
+        self.io, self.device = io, device
+        self.d_model, self.d_inner = d_model, self.scan.d_inner
+        self._ws = {}
+
+    def _proj(self, X2, u2, stream):
+        rows = X2.shape[0]
+        d = self.gate.dims(rows)
+        ws = self._ws.get(rows)
+        need = abi.sambay_in_proj_workspace(d, rows)
+        if ws is None or ws.numel() < need:
+            ws = workspace(need, self.device)
+            self._ws[rows] = ws
+        abi.sambay_in_proj(d, rows, X2, self.W_in, u2, ws, stream)
+
+    def prefill(self, X, ssm_state=None, conv_state=None, fresh=None, stream=None):
+        """X [B, L, Dm] -> (out [B, L, Dm], M [B, L, Di], ssm_state, conv_state)."""
+        B, L, Dm = X.shape
+        X2 = X.reshape(B * L, Dm)
+        u = torch.empty(B, L, self.d_inner, dtype=X.dtype, device=X.device)
+        self._proj(X2, u.view(B * L, self.d_inner), stream)
+        M, h, cs = self.scan.prefill(u, ssm_state, conv_state, fresh=fresh, stream=stream)
+        out = self.gate.forward(X2, M.view(B * L, self.d_inner), residual=True, stream=stream)
+        return out.view(B, L, Dm), M, h, cs
+
+    def step(self, x_t, ssm_state, conv_state, stream=None):
+        """x_t [B, Dm] -> (out_t [B, Dm], m_t [B, Di]); states updated in place."""
+        u_t = torch.empty(x_t.shape[0], self.d_inner, dtype=x_t.dtype, device=x_t.device)
+        self._proj(x_t, u_t, stream)
+        m_t = self.scan.step(u_t, ssm_state, conv_state, stream=stream)
+        out = self.gate.step(x_t, m_t, residual=True, stream=stream)
+        return out, m_t
+
+
+class MLPMemory:
+    """SambaY-MLP's memory: the SwiGLU hidden activation SiLU(X W_g^T) ⊙ (X W_u^T)."""
+
+    def __init__(self, W_g, W_u, io: int, device="cuda"):
+        self.W_g = to_device(W_g, io, device)
+        self.W_u = to_device(W_u, io, device)
+        self.d_ff, self.d_model = W_g.shape
+        self.io, self.device = io, device
+        self._ws = {}
+
+    def forward(self, X, M=None, stream=None):
+        rows = X.shape[0]
+        if M is None:
+            M = torch.empty(rows, self.d_ff, dtype=X.dtype, device=X.device)
+        d = abi.make_dims(rows, 1, self.d_model, self.d_ff, 16, 4, 4, self.io)
+        ws = self._ws.get(rows)
+        need = abi.sambay_mlp_memory_workspace(d, rows)
+        if ws is None or ws.numel() < need:
+            ws = workspace(need, self.device)
+            self._ws[rows] = ws
+        abi.sambay_mlp_memory(d, rows, X, self.W_g, self.W_u, M, ws, stream)
+        return M

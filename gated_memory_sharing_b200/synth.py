@@ -17,6 +17,8 @@ Recipe (one NumPy ``Generator(PCG64)`` per tensor name, seeded from
                        so that softplus(dt_bias) lies in [1e-3, 1e-1] (float32)
     D [Di]           ~ U(0.5, 1.5)                              (float32)
     M (GMU-only)     ~ N(0, 1)
+    Mamba block      W_in, W_z [Di, Dm] ~ N(0, 1/Dm), W_out [Di, Dm] ~ N(0, 1/Di)
+    SwiGLU MLP       W_g, W_u [Dff, Dm] ~ N(0, 1/Dm)
 
 Tensors of the I/O type are rounded to it once here; the same rounded values
 feed both the oracle (widened to float64) and the CUDA path.
@@ -61,6 +63,9 @@ WORKLOADS = {
 WORKLOAD_IDS = {name: i for i, name in enumerate(WORKLOADS)}
 DECODE_STEPS = {"decode_b64": 32768, "sharing_b2_l8192": 4096}
 SHARING_LAYERS = 8
+# cross-attention beside the GMU at d_model 2560: 40 query heads of 64, sharing
+# 20 key/value heads (grouped-query attention)
+ATTN_Q_HEADS, ATTN_KV_HEADS, ATTN_HEAD_DIM = 40, 20, 64
 SHARING_DECODE_BATCH = 16
 LONG_PREFILL_CHUNK = 256
 
@@ -130,6 +135,27 @@ def gmu_weights(d: Dims, seed: int, layer: int = 0) -> dict:
     )
 
 
+def mamba_block_weights(d: Dims, seed: int) -> dict:
+    """in_proj's x and z halves and out_proj (stored [Di, Dm], used on the right)."""
+    r = Draws(seed)
+    Di, Dm = d.d_inner, d.d_model
+    return dict(
+        W_in=to_io(r.normal("W_in", (Di, Dm), 1.0 / np.sqrt(Dm)), d.io),
+        W_z=to_io(r.normal("W_z", (Di, Dm), 1.0 / np.sqrt(Dm)), d.io),
+        W_out=to_io(r.normal("W_out", (Di, Dm), 1.0 / np.sqrt(Di)), d.io),
+    )
+
+
+def mlp_weights(d: Dims, seed: int, d_ff=None) -> dict:
+    """A SwiGLU MLP's gate and up projections, [Dff, Dm] each."""
+    r = Draws(seed)
+    Df = d.d_inner if d_ff is None else d_ff
+    return dict(
+        W_g=to_io(r.normal("W_g", (Df, d.d_model), 1.0 / np.sqrt(d.d_model)), d.io),
+        W_u=to_io(r.normal("W_u", (Df, d.d_model), 1.0 / np.sqrt(d.d_model)), d.io),
+    )
+
+
 def scan_inputs(d: Dims, seed: int, batch=None, seqlen=None, tag="u") -> np.ndarray:
     b = d.batch if batch is None else batch
     L = d.seqlen if seqlen is None else seqlen
@@ -144,6 +170,14 @@ def gmu_inputs(d: Dims, seed: int, rows=None, tag="X") -> np.ndarray:
 def memory_input(d: Dims, seed: int, rows=None, tag="M") -> np.ndarray:
     T = d.tokens if rows is None else rows
     return to_io(Draws(seed).normal(tag, (T, d.d_inner)), d.io)
+
+
+def attention_inputs(batch: int, kv_len: int, q_heads: int, kv_heads: int, head_dim: int, seed: int):
+    """q [B, Hq, dh] and the KV cache K, V [B, N, Hkv, dh], N(0, 1), bf16-rounded."""
+    r = Draws(seed)
+    return (round_bf16(r.normal("q", (batch, q_heads, head_dim))),
+            round_bf16(r.normal("K", (batch, kv_len, kv_heads, head_dim))),
+            round_bf16(r.normal("V", (batch, kv_len, kv_heads, head_dim))))
 
 
 def workload(name: str):

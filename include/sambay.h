@@ -188,6 +188,48 @@ SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const v
                        const void* W1, const void* W2, const void* residual, void* Y,
                        void* ws, size_t ws_bytes, sambay_stream_t stream);
 
+/*
+ * sambay_in_proj - the scan branch of the Mamba block's input projection
+ * [MAMBA] section 3.4: u = X W_in^T, the input of sambay_scan_prefill /
+ * sambay_scan_step.  With it the whole Mamba layer whose readout is the
+ * memory M runs from its input X [FRAME] (the Samba self-decoder's SSM
+ * layers):
+ *     u = sambay_in_proj(X, W_in);   M = sambay_scan_prefill(u)  (pre-gate y)
+ *     out = gmu_forward(X, M, W_z, W_out, residual = X)
+ * since the block's gated output (y ⊙ SiLU(X W_z^T)) W_out is the GMU's
+ * computation with W1 = W_z (the z half of in_proj) and W2 = W_out (out_proj's
+ * weight, [Di, Dm], multiplying on the right).
+ *
+ *   X [rows, Dm] io;  W_in [Di, Dm] io (used transposed);  u [rows, Di] io out
+ *   (must not alias X).  ws: >= sambay_in_proj_workspace(dims, rows) (the
+ *   K-split tail partials of a bf16 GEMM of more than 256 rows; else 0).
+ * Up to 256 rows (decode) W_in streams once through the swap-AB decode GEMM.
+ */
+SAMBAY_API size_t sambay_in_proj_workspace(const sambay_dims* dims, int64_t rows);
+SAMBAY_API sambay_status sambay_in_proj(const sambay_dims* dims, int64_t rows, const void* X,
+                                        const void* W_in, void* u, void* ws, size_t ws_bytes,
+                                        sambay_stream_t stream);
+
+/*
+ * sambay_mlp_memory - the memory of SambaY-MLP ([Notes] 实验关键数据 >
+ * 消融实验, row SambaY-MLP: the GMUs gate an MLP representation instead of the
+ * SSM readout): the hidden activation of a SwiGLU MLP,
+ *     M = SiLU(X W_g^T) ⊙ (X W_u^T),
+ * which gmu_forward / gmu_step then take in place of the scan readout.
+ * dims->d_inner is the MLP width Dff, dims->d_model the input width.
+ *
+ *   X [rows, Dm] io;  W_g, W_u [Dff, Dm] io (used transposed);
+ *   M [rows, Dff] io out (must not alias X);
+ *   ws: >= sambay_mlp_memory_workspace(dims, rows) (X W_u^T, then the K-split
+ *   tail partials as in sambay_in_proj).
+ * Two tensor-core GEMMs: X W_u^T, then X W_g^T with SiLU and the product with
+ * X W_u^T fused into its epilogue (the GMU gate GEMM's epilogue).
+ */
+SAMBAY_API size_t sambay_mlp_memory_workspace(const sambay_dims* dims, int64_t rows);
+SAMBAY_API sambay_status sambay_mlp_memory(const sambay_dims* dims, int64_t rows, const void* X,
+                                           const void* W_g, const void* W_u, void* M, void* ws,
+                                           size_t ws_bytes, sambay_stream_t stream);
+
 /* Weights of one Gated Memory Unit layer (device pointers, [Di, Dm] io each). */
 typedef struct {
   const void* W1; /* used as W1^T: X W1^T maps Dm -> Di   */
@@ -236,6 +278,38 @@ SAMBAY_API sambay_status sambay_gmu_step_stall_test(const sambay_dims* dims, int
                                                     const void* residual, void* Y, void* ws,
                                                     size_t ws_bytes, uint64_t wait_limit_cycles,
                                                     sambay_stream_t stream);
+
+/* Sizes of a cross-attention decode.  Tensors are bfloat16. */
+typedef struct {
+  int32_t batch;      /* B sequences, one query token each                  */
+  int32_t kv_len;     /* N cached tokens per sequence                        */
+  int32_t q_heads;    /* Hq query heads                                      */
+  int32_t kv_heads;   /* Hkv key/value heads; Hq / Hkv <= 16 share one       */
+  int32_t head_dim;   /* dh: 64 or 128                                       */
+} sambay_attn_dims;
+
+/*
+ * sambay_cross_attn_decode - one decoded token per sequence attending over
+ * the single KV cache that the self-decoder's full-attention layer wrote once
+ * [FRAME] (the cross-decoder's cross-attention layers, the ones the GMU does
+ * not replace), i.e. the O(d_kv N) memory-per-token counterpart of gmu_step's
+ * O(d_h):
+ *     out[b, h] = sum_j softmax_j(scale q[b, h] . K[b, j, h / G]) V[b, j, h / G]
+ * with G = Hq / Hkv (consecutive query heads share a KV head).
+ *
+ *   q [B, Hq, dh], K and V [B, N, Hkv, dh] (token-major), out [B, Hq, dh],
+ *   all bf16 (out must not alias the inputs); scale > 0, or 0 for
+ *   1 / sqrt(dh).  ws: >= sambay_cross_attn_decode_workspace(dims) (the
+ *   partial outputs of a KV range split over several CTAs; 0 when the
+ *   sequences and heads alone fill the GPU).
+ * Split-KV: each CTA streams a range of one (sequence, KV head)'s tokens
+ * once, with an online softmax and fp32 accumulation; ranges are combined in
+ * a fixed order.
+ */
+SAMBAY_API size_t sambay_cross_attn_decode_workspace(const sambay_attn_dims* dims);
+SAMBAY_API sambay_status sambay_cross_attn_decode(const sambay_attn_dims* dims, const void* q,
+                                                  const void* K, const void* V, void* out, float scale,
+                                                  void* ws, size_t ws_bytes, sambay_stream_t stream);
 
 /*
  * sambay_scan_step_noalloc - sambay_scan_step for callers that cannot

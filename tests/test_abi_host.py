@@ -85,6 +85,32 @@ def test_decode_step_argument_errors(lib):
     assert e.value.code == 1
 
 
+def test_cross_attn_argument_errors(lib):
+    p = _FakePtr(0x10000)
+    ok = abi.AttnDims(2, 1000, 4, 2, 64)
+    # 4 (sequence, KV head) pairs: the KV range splits over CTAs, whose partials need scratch
+    assert abi.sambay_cross_attn_decode_workspace(ok) > 0
+    assert abi.sambay_cross_attn_decode_workspace(abi.AttnDims(64, 2048, 40, 20, 64)) == 0
+    for bad, code in ((abi.AttnDims(2, 100, 4, 2, 96), 2),     # head size
+                      (abi.AttnDims(2, 100, 6, 4, 64), 2),     # heads not grouped evenly
+                      (abi.AttnDims(2, 100, 34, 2, 64), 2),    # more than 16 query heads per KV head
+                      (abi.AttnDims(0, 100, 4, 2, 64), 1)):
+        assert abi.sambay_cross_attn_decode_workspace(bad) == 0
+        with pytest.raises(abi.SambayError) as e:
+            abi.sambay_cross_attn_decode(bad, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000), 0.0, p, 0)
+        assert e.value.code == code
+    with pytest.raises(abi.SambayError) as e:     # NULL input
+        abi.sambay_cross_attn_decode(ok, None, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000), 0.0, p, 0)
+    assert e.value.code == 1
+    with pytest.raises(abi.SambayError) as e:     # NaN scale
+        abi.sambay_cross_attn_decode(ok, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                                     float("nan"), p, 0)
+    assert e.value.code == 1
+    with pytest.raises(abi.SambayError) as e:     # workspace too small
+        abi.sambay_cross_attn_decode(ok, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000), 0.0, p, 0)
+    assert e.value.code == 3
+
+
 def test_status_strings_and_version(lib):
     assert abi.sambay_version() == "0.1.0"
     assert abi.sambay_status_string(0) == "ok"
