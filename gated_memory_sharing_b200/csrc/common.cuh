@@ -87,6 +87,31 @@ __device__ __forceinline__ float4 ldcg_or_zero(const float* p, bool pred) {
   return v;
 }
 
+// Loads from shared memory by a shared-space address (ld.shared), whatever
+// the compiler can prove about the generic pointer: a generic load may be
+// ordered behind the thread's earlier global stores, a shared one is not.
+__device__ __forceinline__ uint32_t shared_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ float4 ld_shared_f4(const void* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(shared_addr(p))
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_shared_f32(const void* p) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(shared_addr(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_shared_bf16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(shared_addr(p)) : "memory");
+  return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
 // Pack / unpack helpers for 16-byte vector access.
 union Pack16 {
   uint4 u;

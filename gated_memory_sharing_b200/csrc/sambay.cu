@@ -177,6 +177,8 @@ struct StepPlan {
   bool ok = false;
   int chan = 0, nslice = 0, group = 0, Rp = 0;
   size_t smem = 0;
+  bool fused = false;      // one cooperative kernel (batch <= 64 and its layout fits)
+  size_t fused_smem = 0;
 };
 
 StepPlan step_plan(const sambay_dims* d) {
@@ -195,6 +197,14 @@ StepPlan step_plan(const sambay_dims* d) {
   sp.group = group;
   sp.smem = static_cast<size_t>(ly.bytes);
   sp.ok = true;
+  if (d->batch <= sambay::step::kMaxGroup) {
+    const int ldx = d->dt_rank + 2 * d->d_state;
+    const sambay::step::FusedStepLayout fl(sp.chan, d->batch, sp.Rp, ldx, sp.nslice);
+    if (fl.bytes <= kMaxDynSmemBytes) {
+      sp.fused = true;
+      sp.fused_smem = static_cast<size_t>(fl.bytes);
+    }
+  }
   return sp;
 }
 
@@ -204,9 +214,9 @@ struct ScanWs {
 };
 
 // Scratch of the bf16 decode step: conv output, x_proj partials per slice,
-// the split delta and B | C.
+// the split delta, B | C, and the single-kernel form's meeting words.
 struct StepWs {
-  size_t uc, part, dts, bc, total;
+  size_t uc, part, dts, bc, bar, total;
 };
 
 StepWs step_ws_layout(const sambay_dims* d, const StepPlan& sp) {
@@ -217,6 +227,7 @@ StepWs step_ws_layout(const sambay_dims* d, const StepPlan& sp) {
   w.part = off; off += round256(static_cast<size_t>(sp.nslice) * ldx * B * 4);
   w.dts = off;  off += round256(2 * B * static_cast<size_t>(sp.Rp) * 2);
   w.bc = off;   off += round256(B * 2 * d->d_state * 4);
+  w.bar = off;  off += round256(static_cast<size_t>(sambay::step::fused_bar_words(sp.nslice)) * 8);
   w.total = off;
   return w;
 }
@@ -791,9 +802,11 @@ sambay_status scan_step_fused(int dev, int sms, const sambay_scan_weights* w, co
   auto kproj = sambay::step::step_proj_kernel;
   auto kred = sambay::step::step_reduce_kernel;
   auto kscan = sambay::step::step_scan_kernel;
+  auto kfused = sambay::step::step_fused_kernel;
   static bool attr_set[kMaxDevices] = {};
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kscan, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kscan, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kfused, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmemBytes) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
     attr_set[dev] = true;
   }
@@ -817,6 +830,8 @@ sambay_status scan_step_fused(int dev, int sms, const sambay_scan_weights* w, co
   p.part = reinterpret_cast<float*>(ws + L.part);
   p.dts = reinterpret_cast<bf16*>(ws + L.dts);
   p.bc = reinterpret_cast<float*>(ws + L.bc);
+  p.bar = reinterpret_cast<unsigned long long*>(ws + L.bar);
+  p.wait_limit = sambay::tc::kWaitCycles;
   p.B = d->batch;
   p.Di = d->d_inner;
   p.R = d->dt_rank;
@@ -825,6 +840,36 @@ sambay_status scan_step_fused(int dev, int sms, const sambay_scan_weights* w, co
   p.chan = sp.chan;
   p.nslice = sp.nslice;
   p.group = sp.group;
+  if (sp.fused && sp.nslice <= sms && sp.nslice <= sambay::step::kMaxMeetCtas) {
+    // one kernel; cooperative, so its CTAs (one per slice) are all resident at
+    // once, which its grid-wide meeting points need.  The state h viewed as
+    // [B][Di / 8][128 floats]: a CTA's slice is the box {128, chan / 8, B}.
+    SAMBAY_MAX_CARVEOUT(kfused, dev);
+    EncodeTiledFn fn = encode_fn();
+    CUtensorMap hmap;
+    {
+      const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(d->d_inner / 8), static_cast<cuuint64_t>(d->batch)};
+      const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(d->d_inner) * 64};
+      const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(sp.chan / 8), static_cast<cuuint32_t>(d->batch)};
+      const cuuint32_t es[3] = {1, 1, 1};
+      if (!fn || fn(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ssm_state, dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return SAMBAY_ERR_CUDA;
+    }
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(sp.nslice);
+    lc.blockDim = dim3(sambay::step::kFusedThreads);
+    lc.dynamicSmemBytes = sp.fused_smem;
+    lc.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    ProfScope ps("step_fused", st);
+    return cudaLaunchKernelEx(&lc, kfused, p, hmap) == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
+  }
   const dim3 grid(sp.nslice, (d->batch + sp.group - 1) / sp.group);
   const dim3 block(sambay::step::kThreads);
   {

@@ -42,6 +42,8 @@
 // both operands, which makes each pair of registers one 8-byte load.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace sambay {
@@ -73,6 +75,8 @@ struct StepParams {
   float* part;            // [nslice][ldx][B]   x_proj partial sums
   bf16* dts;              // [2B][Rp]           delta split pair (row 2s: hi, 2s + 1: lo)
   float* bc;              // [B][2N]            B | C
+  unsigned long long* bar;  // [1 + 2 * nslice]  step_fused: generation word, arrival flags
+  unsigned long long wait_limit;  // step_fused: bounded-wait limit (clock64 cycles)
   int B, Di, R, Rp, ldx;
   int chan, nslice;       // channels per slice (multiple of 8, <= kMaxChan), slices
   int group;              // sequences per CTA (<= kMaxGroup)
@@ -429,6 +433,484 @@ __global__ void __launch_bounds__(kThreads, 1) step_scan_kernel(const StepParams
     if (q == 0) p.m_t[hc] = __float2bfloat16_rn(fmaf(d_s[c], uu, y));
     c += kThreads / 4;
     while (c >= chan) { c -= chan; ++s; }
+  }
+}
+
+// ------------------------------------------------------------------ step_fused
+
+// The same step as ONE kernel when every slice fits one CTA of all sequences
+// (batch <= 64) and the slices fit the GPU at one CTA per SM: launched
+// cooperatively, so all CTAs are resident together, and the two points where
+// the step needs every slice's result (the x_proj sum over channels, then its
+// use by every slice) are grid-wide meeting points instead of kernel
+// boundaries.  The slice's state arrives as one tensor copy and its W_dt, A,
+// b_dt and D slices by cp.async, both issued behind the conv's own loads and
+// landing under the conv, the partial x_proj and both meetings.
+//
+//   phase 0   conv of the slice (uc stays in shared memory), partial x_proj
+//             sums part[slice][seq][j] (m16n8k16)
+//   meet 1
+//   phase 1   CTA k sums outputs [k per, (k + 1) per) of [delta | B | C] over
+//             the slices: warp w adds slices [w spw, (w + 1) spw) in order,
+//             then the warps' sums are added in warp order (a fixed order)
+//   meet 2
+//   phase 2   dt = softplus(delta W_dt^T + b_dt) for the slice (m16n8k16), the
+//             state update and readout
+//
+// Meeting points: after a CTA barrier, CTA b stores `target` into its own
+// flag with release semantics (cumulative over the CTA's writes ordered
+// before it by the barrier), and one warp of every CTA reads all flags
+// (relaxed) until each holds `target`, then fences (acquire) before the CTA
+// barrier that releases the other warps.  Each flag has a 128-byte line of
+// its own, so the reads spread over the L2.  `target` = the generation word +
+// 1; CTA 0 advances the generation word after the second meeting, when every
+// CTA has read it, so flags left by an earlier call never match whatever the
+// words held before.  Waits are bounded (wait_limit cycles); a CTA whose wait
+// runs out records the timeout status, lets its copies in flight land and
+// returns.
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kMaxSpw = 10;       // slices per warp in phase 1 (148 slices / 16 warps)
+constexpr int kFlagStride = 16;   // u64 words between flags (one 128-byte line each)
+constexpr int kMaxMeetCtas = 160; // CTAs a meeting point's polling warp covers (5 flags per lane)
+static_assert(kMaxGroup * (kMaxChan / 8) <= kFusedThreads, "one conv item per thread");
+
+__host__ __device__ constexpr int fused_per_cta(int ldx, int B, int nslice) {
+  return (ldx * B + nslice - 1) / nslice;
+}
+__host__ __device__ constexpr int max_i(int a, int b) { return a > b ? a : b; }
+// meeting words: generation (own line), then two arrays of nslice flags
+__host__ __device__ constexpr long long fused_bar_words(int nslice) {
+  return static_cast<long long>(kFlagStride) * (1 + 2 * nslice);
+}
+
+// Dynamic shared memory of step_fused (byte offsets).
+struct FusedStepLayout {
+  int mtl, dp, per;
+  int h, w, a, bias, dv, uc, bc, un, misc, bytes;
+  __host__ __device__ FusedStepLayout(int chan, int B, int Rp, int ldx, int nslice) {
+    mtl = (chan + 15) / 16;
+    dp = frag_pitch(Rp);
+    per = fused_per_cta(ldx, B, nslice);
+    h = 0;                                             // f32 [B][chan][N]
+    w = h + B * chan * kStateN * 4;                    // bf16 [mtl*16][dp] W_dt rows
+    a = w + round_up(mtl * 16 * dp * 2, 16);           // f32 [chan][N]
+    bias = a + chan * kStateN * 4;                     // f32 [chan]
+    dv = bias + round_up(chan * 4, 16);                // f32 [chan]
+    uc = dv + round_up(chan * 4, 16);                  // f32 [B][chan]
+    bc = uc + round_up(B * chan * 4, 16);              // f32 [B][2N]
+    un = bc + B * 2 * kStateN * 4;                     // one of, by phase:
+    const int ucs_b = 2 * round_up(B, 4) * kUcsPitch * 2;   //   bf16 conv output split pair
+    const int red_b = kFusedWarps * per * 4;                 //   f32 [warps][per] phase-1 sums
+    const int dt_b = B * chan * 4;                           //   f32 [B][chan] dt
+    misc = un + round_up(max_i(ucs_b, max_i(red_b, dt_b)), 16);   // u64 generation, int ok, u64 mbarrier
+    bytes = misc + 24;
+  }
+};
+
+// mbarrier and bulk-copy glue (non-multicast forms only)
+__device__ __forceinline__ uint32_t sh_addr(const void* ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+__device__ __forceinline__ void mb_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sh_addr(bar)), "r"(count));
+}
+__device__ __forceinline__ void mb_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sh_addr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mb_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(ok)
+      : "r"(sh_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait for phase `parity` of `bar`
+__device__ __forceinline__ bool mb_wait(uint64_t* bar, uint32_t parity, unsigned long long limit) {
+  if (mb_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mb_try_wait(bar, parity))
+    if (static_cast<unsigned long long>(clock64() - t0) > limit) return false;
+  return true;
+}
+// 3-D tensor copy global -> shared completing on `bar` (no multicast)
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          sh_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(sh_addr(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* ptr) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* ptr, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");
+}
+
+// Grid-wide meeting point (see above).  Every thread of the CTA returns the
+// same answer: false if some flag did not arrive in time.
+__device__ bool grid_meet(unsigned long long* flags, unsigned long long target, unsigned long long limit,
+                          int* ok_s) {
+  __syncthreads();   // the CTA's writes before the release below (cumulative)
+  if (threadIdx.x == 0) st_release_u64(flags + static_cast<long long>(blockIdx.x) * kFlagStride, target);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const long long t0 = clock64();
+    while (true) {
+      // all of the lane's flags (at most 5 of 148) read at once, then compared
+      unsigned long long v[5];
+#pragma unroll
+      for (int k = 0; k < 5; ++k) {
+        const int i = lane + 32 * k;
+        v[k] = i < static_cast<int>(gridDim.x) ? ld_relaxed_u64(flags + static_cast<long long>(i) * kFlagStride)
+                                                : target;
+      }
+      bool mine = true;
+#pragma unroll
+      for (int k = 0; k < 5; ++k) mine = mine && v[k] == target;
+      if (__all_sync(0xffffffffu, mine)) break;
+      if (static_cast<unsigned long long>(clock64() - t0) > limit) {
+        if (lane == 0) {
+          *reinterpret_cast<volatile int*>(ok_s) = 0;
+          record_status(kStatusTimeout);
+        }
+        break;
+      }
+      __nanosleep(32);
+    }
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");   // later reads of other CTAs' data see their writes
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int*>(ok_s) != 0;
+}
+
+__global__ void __launch_bounds__(kFusedThreads, 1) step_fused_kernel(const StepParams p,
+                                                                     const __grid_constant__ CUtensorMap hmap) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int chan = p.chan, c0 = blockIdx.x * chan, B = p.B;
+  const int Di = p.Di, R = p.R, Rp = p.Rp, ldx = p.ldx, nslice = p.nslice;
+  const FusedStepLayout ly(chan, B, Rp, ldx, nslice);
+  float* h_s = reinterpret_cast<float*>(smem + ly.h);
+  bf16* w_s = reinterpret_cast<bf16*>(smem + ly.w);
+  float* a_s = reinterpret_cast<float*>(smem + ly.a);
+  float* bias_s = reinterpret_cast<float*>(smem + ly.bias);
+  float* d_s = reinterpret_cast<float*>(smem + ly.dv);
+  float* uc_s = reinterpret_cast<float*>(smem + ly.uc);
+  float* bc_s = reinterpret_cast<float*>(smem + ly.bc);
+  bf16* ucs = reinterpret_cast<bf16*>(smem + ly.un);
+  float* red_s = reinterpret_cast<float*>(smem + ly.un);
+  float* dt_s = reinterpret_cast<float*>(smem + ly.un);
+  unsigned long long& gen_s = *reinterpret_cast<unsigned long long*>(smem + ly.misc);
+  int& ok_s = *reinterpret_cast<int*>(smem + ly.misc + 8);
+  uint64_t* mb = reinterpret_cast<uint64_t*>(smem + ly.misc + 16);
+  if (tid == 0) {
+    ok_s = 1;
+    gen_s = *reinterpret_cast<volatile unsigned long long*>(p.bar);
+    mb_init(mb, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_smem();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&hmap)) : "memory");
+  }
+  pdl_launch_dependents();
+  __syncthreads();
+
+  // ---- phase 0a: what the conv and the partial x_proj need first, to
+  // registers: the W_x fragments of the warp's first row tile, and the
+  // thread's conv item (8 channels of one sequence; 4 nblk vpc <= 384 items,
+  // at most one per thread)
+  const int kc = round_up(chan, 16), ksteps = kc / 16;
+  const int mtiles = (ldx + 15) / 16;
+  auto load_wx = [&](int mt, uint32_t (&a)[3][4]) {
+#pragma unroll
+    for (int ks = 0; ks < 3; ++ks) {
+      const int col = c0 + ks * 16 + 4 * t;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int j = mt * 16 + g + 8 * half;
+        uint2 v = make_uint2(0u, 0u);
+        if (ks < ksteps && j < ldx && col + 3 < Di)
+          v = *reinterpret_cast<const uint2*>(p.x_proj_w + static_cast<long long>(j) * Di + col);
+        a[ks][half] = v.x;          // logical k 2t, 2t+1
+        a[ks][2 + half] = v.y;      // logical k 2t+8, 2t+9
+      }
+    }
+  };
+  uint32_t afr[3][4];
+  if (warp < mtiles) load_wx(warp, afr);
+  const int nblk = (B + 3) / 4;
+  const int vpc = chan / 8;
+  const int cs = tid / vpc, cl = (tid % vpc) * 8;     // conv item: sequence cs, channels cl .. cl+7
+  const bool conv_item = tid < 4 * nblk * vpc;
+  const bool conv_live = conv_item && cs < B;
+  const long long coff = static_cast<long long>(cs) * Di + c0 + cl;
+  Pack16 in, cbias, win[4], wt[4];
+  if (conv_live) {
+    in.u = *reinterpret_cast<const uint4*>(p.u_t + coff);
+    cbias.u = *reinterpret_cast<const uint4*>(p.conv_b + c0 + cl);
+    const uint4* wp = reinterpret_cast<const uint4*>(p.conv_state + coff * kConvK);
+    const uint4* kp = reinterpret_cast<const uint4*>(p.conv_w + static_cast<long long>(c0 + cl) * kConvK);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      win[j].u = wp[j];
+      wt[j].u = kp[j];
+    }
+  }
+
+  // ---- phase 0b, behind those loads: the slice's state as ONE tensor copy
+  // (box {128 floats, chan / 8, B} of h viewed as [B][Di / 8][128]) landing
+  // on `mb`, and the W_dt rows, A, b_dt and D slices (cp.async); all of it
+  // lands while the conv, the x_proj and both meetings run
+  if (tid == 0) {
+    mb_expect_tx(mb, static_cast<uint32_t>(B) * chan * kStateN * 4);
+    tma_load_3d(h_s, &hmap, mb, 0, c0 / 8, 0);
+  }
+  {
+    const int rc = R / 8;
+    for (int i = tid; i < chan * rc; i += kFusedThreads) {
+      const int r = i / rc, k = i % rc;
+      cp_async16(w_s + r * ly.dp + 8 * k, p.dt_proj_w + static_cast<long long>(c0 + r) * R + 8 * k);
+    }
+    for (int i = tid; i < chan * kStateN / 4; i += kFusedThreads)
+      cp_async16(a_s + 4 * i, p.A + static_cast<long long>(c0) * kStateN + 4 * i);
+    for (int i = tid; i < chan / 4; i += kFusedThreads) {
+      cp_async16(bias_s + 4 * i, p.dt_bias + c0 + 4 * i);
+      cp_async16(d_s + 4 * i, p.D + c0 + 4 * i);
+    }
+    cp_async_commit();
+  }
+  for (int i = tid; i < (ly.mtl * 16 - chan) * ly.dp; i += kFusedThreads)   // W_dt rows past the slice
+    w_s[chan * ly.dp + i] = __float2bfloat16_rn(0.0f);
+  for (int i = tid; i < chan * (Rp - R); i += kFusedThreads)                   // k padding
+    w_s[(i / (Rp - R)) * ly.dp + R + i % (Rp - R)] = __float2bfloat16_rn(0.0f);
+
+  // ---- phase 0c: conv + SiLU (window shifted in place)
+  if (conv_item) {
+    float y[8];
+    if (conv_live) {
+      bf16* wv = reinterpret_cast<bf16*>(win);            // [8 channels][K], oldest first
+      const bf16* kv = reinterpret_cast<const bf16*>(wt);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+#pragma unroll
+        for (int k = 0; k < kConvK - 1; ++k) wv[e * kConvK + k] = wv[e * kConvK + k + 1];
+        wv[e * kConvK + kConvK - 1] = in.h[e];
+        float acc = __bfloat162float(cbias.h[e]);
+#pragma unroll
+        for (int k = 0; k < kConvK; ++k)
+          acc = fmaf(__bfloat162float(kv[e * kConvK + k]), __bfloat162float(wv[e * kConvK + k]), acc);
+        y[e] = silu(acc);
+      }
+      uint4* wp = reinterpret_cast<uint4*>(p.conv_state + coff * kConvK);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wp[j] = win[j].u;
+      float4* us = reinterpret_cast<float4*>(uc_s + cs * chan + cl);
+      us[0] = make_float4(y[0], y[1], y[2], y[3]);
+      us[1] = make_float4(y[4], y[5], y[6], y[7]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = 0.0f;
+    }
+    Pack16 hi, lo;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) split_bf16(y[e], hi.h[e], lo.h[e]);
+    *reinterpret_cast<uint4*>(ucs + (2 * cs) * kUcsPitch + cl) = hi.u;
+    *reinterpret_cast<uint4*>(ucs + (2 * cs + 1) * kUcsPitch + cl) = lo.u;
+  }
+  for (int it = tid; it < 8 * nblk * (kc - chan); it += kFusedThreads) {   // k padding
+    const int r = it / (kc - chan), c = chan + it % (kc - chan);
+    ucs[r * kUcsPitch + c] = __float2bfloat16_rn(0.0f);
+  }
+  __syncthreads();
+
+  // ---- phase 0d: partial x_proj D[j][n] = sum_{c in slice} W_x[j][c] ucs[n][c],
+  // stored as part[slice][seq][j]
+  for (int mt = warp; mt < mtiles; mt += kFusedWarps) {
+    if (mt != warp) load_wx(mt, afr);
+    float acc[16][4];
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.0f;
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) {
+      if (nb >= nblk) break;
+#pragma unroll
+      for (int ks = 0; ks < 3; ++ks) {
+        if (ks >= ksteps) break;
+        const uint2 b = lds64(ucs + (8 * nb + g) * kUcsPitch + ks * 16 + 4 * t);
+        mma16816(acc[nb], afr[ks][0], afr[ks][1], afr[ks][2], afr[ks][3], b.x, b.y);
+      }
+    }
+    float* part = p.part + static_cast<long long>(blockIdx.x) * B * ldx;
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) {            // D[j][8nb + 2t + {0, 1}]: (hi, lo) of sequence 4nb + t
+      if (nb >= nblk) break;
+      const int s = 4 * nb + t;
+      if (s >= B) continue;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int j = mt * 16 + g + 8 * half;
+        if (j < ldx) part[s * ldx + j] = acc[nb][2 * half] + acc[nb][2 * half + 1];
+      }
+    }
+  }
+
+  const unsigned long long target = gen_s + 1;
+  unsigned long long* flags1 = p.bar + kFlagStride;
+  unsigned long long* flags2 = flags1 + static_cast<long long>(nslice) * kFlagStride;
+  if (!grid_meet(flags1, target, p.wait_limit, &ok_s)) {
+    cp_async_wait<0>();
+    mb_wait(mb, 0, p.wait_limit);   // copies into this CTA's shared memory land before it leaves
+    return;
+  }
+
+  // ---- phase 1: outputs [o0, o1) of [delta | B | C] (o = seq * ldx + j);
+  // every load of a lane (kRounds rounds of 32 outputs x its slices) in flight
+  // at once, then the adds in slice order
+  {
+    constexpr int kRounds = 4;
+    const int per = ly.per, total = ldx * B;
+    const int o0 = blockIdx.x * per, o1 = min(total, o0 + per);
+    const int spw = (nslice + kFusedWarps - 1) / kFusedWarps;
+    const int sl0 = warp * spw, sl1 = min(nslice, sl0 + spw);
+    const long long sstride = static_cast<long long>(ldx) * B;
+    for (int r0 = 0; r0 * 32 < per; r0 += kRounds) {
+      float x[kRounds][kMaxSpw];
+#pragma unroll
+      for (int rr = 0; rr < kRounds; ++rr) {
+        const int oi = (r0 + rr) * 32 + lane, o = o0 + oi;
+        const bool valid = oi < per && o < o1;
+#pragma unroll
+        for (int k = 0; k < kMaxSpw; ++k)
+          x[rr][k] = (valid && sl0 + k < sl1) ? __ldcg(p.part + (sl0 + k) * sstride + o) : 0.0f;
+      }
+#pragma unroll
+      for (int rr = 0; rr < kRounds; ++rr) {
+        const int oi = (r0 + rr) * 32 + lane;
+        float acc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kMaxSpw; ++k) acc += x[rr][k];
+        if (oi < per) red_s[warp * per + oi] = acc;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < o1 - o0; i += kFusedThreads) {
+      float acc = 0.0f;
+      for (int w2 = 0; w2 < kFusedWarps; ++w2) acc += red_s[w2 * per + i];
+      const int o = o0 + i, s = o / ldx, j = o % ldx;
+      if (j < R) {
+        bf16 hi, lo;
+        split_bf16(acc, hi, lo);
+        p.dts[(2LL * s) * Rp + j] = hi;
+        p.dts[(2LL * s + 1) * Rp + j] = lo;
+      } else {
+        p.bc[static_cast<long long>(s) * 2 * kStateN + (j - R)] = acc;
+      }
+    }
+    if (blockIdx.x == 0)
+      for (int i = tid; i < 2 * B * (Rp - R); i += kFusedThreads)
+        p.dts[(i / (Rp - R)) * Rp + R + i % (Rp - R)] = __float2bfloat16_rn(0.0f);
+  }
+
+  if (!grid_meet(flags2, target, p.wait_limit, &ok_s)) {
+    cp_async_wait<0>();
+    mb_wait(mb, 0, p.wait_limit);
+    return;
+  }
+  if (blockIdx.x == 0 && tid == 0) *reinterpret_cast<volatile unsigned long long*>(p.bar) = target;
+
+  // ---- phase 2: B | C of every sequence, delta fragments, dt, state update
+  for (int i = tid; i < B * 2 * kStateN / 4; i += kFusedThreads) cp_async16(bc_s + 4 * i, p.bc + 4 * i);
+  cp_async_commit();
+  const int kst = Rp / 16;
+  uint32_t bfr[14][2];
+  {
+    const int row = 8 * warp + g;                       // split-pair row of n-block `warp`
+    const bool live = warp < nblk && row < 2 * B;
+#pragma unroll
+    for (int ks = 0; ks < 14; ++ks) {
+      uint2 v = make_uint2(0u, 0u);
+      if (live && ks < kst)
+        v = __ldcg(reinterpret_cast<const uint2*>(p.dts + static_cast<long long>(row) * Rp + ks * 16 + 4 * t));
+      bfr[ks][0] = v.x;
+      bfr[ks][1] = v.y;
+    }
+  }
+  cp_async_wait<0>();
+  if (!mb_wait(mb, 0, p.wait_limit)) {
+    *reinterpret_cast<volatile int*>(&ok_s) = 0;
+    record_status(kStatusTimeout);
+  }
+  __syncthreads();
+  if (!*reinterpret_cast<volatile int*>(&ok_s)) return;
+  if (warp < nblk) {          // n-block `warp`, the slice's (at most 3) row tiles side by side
+    float acc[3][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 14; ++ks) {
+      if (ks >= kst) break;
+#pragma unroll
+      for (int mt = 0; mt < 3; ++mt) {
+        if (mt >= ly.mtl) break;
+        const uint2 a_lo = lds64(w_s + (mt * 16 + g) * ly.dp + ks * 16 + 4 * t);
+        const uint2 a_hi = lds64(w_s + (mt * 16 + g + 8) * ly.dp + ks * 16 + 4 * t);
+        mma16816(acc[mt], a_lo.x, a_hi.x, a_lo.y, a_hi.y, bfr[ks][0], bfr[ks][1]);
+      }
+    }
+    const int s = 4 * warp + t;
+    if (s < B) {
+#pragma unroll
+      for (int mt = 0; mt < 3; ++mt) {
+        if (mt >= ly.mtl) break;
+        const int c = mt * 16 + g;
+        if (c < chan) dt_s[s * chan + c] = softplus(acc[mt][0] + acc[mt][1] + bias_s[c]);
+        if (c + 8 < chan) dt_s[s * chan + c + 8] = softplus(acc[mt][2] + acc[mt][3] + bias_s[c + 8]);
+      }
+    }
+  }
+  __syncthreads();
+
+  // state update and readout: thread (row, c, quarter q) owns states 4q ..
+  // 4q+3 of channel c for sequences row, row + rows, ...; chan * 4 threads
+  // per row (a multiple of 32: warps never straddle rows), the quarters of a
+  // channel on 4 consecutive lanes
+  const int per_row = chan * 4, rows = kFusedThreads / per_row;
+  if (tid < rows * per_row) {
+    const int row = tid / per_row, c = (tid % per_row) >> 2, q = tid & 3;
+    const float4 av = *reinterpret_cast<const float4*>(a_s + c * kStateN + 4 * q);
+    const float4 al = make_float4(av.x * kLog2e, av.y * kLog2e, av.z * kLog2e, av.w * kLog2e);
+    const float dd = d_s[c];
+#pragma unroll 2
+    for (int s = row; s < B; s += rows) {
+      const float4 hv = ld_shared_f4(h_s + (s * chan + c) * kStateN + 4 * q);
+      const float d = ld_shared_f32(dt_s + s * chan + c);
+      const float uu = ld_shared_f32(uc_s + s * chan + c);
+      const float4 bv = ld_shared_f4(bc_s + s * 2 * kStateN + 4 * q);
+      const float4 cv = ld_shared_f4(bc_s + s * 2 * kStateN + kStateN + 4 * q);
+      const float du = d * uu;
+      float4 hn;
+      hn.x = fmaf(ex2_approx(d * al.x), hv.x, du * bv.x);
+      hn.y = fmaf(ex2_approx(d * al.y), hv.y, du * bv.y);
+      hn.z = fmaf(ex2_approx(d * al.z), hv.z, du * bv.z);
+      hn.w = fmaf(ex2_approx(d * al.w), hv.w, du * bv.w);
+      float y = cv.x * hn.x;
+      y = fmaf(cv.y, hn.y, y);
+      y = fmaf(cv.z, hn.z, y);
+      y = fmaf(cv.w, hn.w, y);
+      y += __shfl_xor_sync(0xffffffffu, y, 1);
+      y += __shfl_xor_sync(0xffffffffu, y, 2);
+      const long long hc = static_cast<long long>(s) * Di + c0 + c;
+      *reinterpret_cast<float4*>(p.h + hc * kStateN + 4 * q) = hn;
+      if (q == 0) p.m_t[hc] = __float2bfloat16_rn(fmaf(dd, uu, y));
+    }
   }
 }
 

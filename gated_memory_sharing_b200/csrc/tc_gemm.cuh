@@ -1108,36 +1108,37 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     // those stores) each CTA sums its rows [split * R, +R) locally, in split
     // order, and applies the final op.  Nothing touches a peer's shared
     // memory after the barrier, so no second barrier is needed before exit.
-    // Thread: 4 consecutive columns of one row, consecutive threads on
-    // consecutive rows.
+    // Thread: row tid % 64 of the CTA's rows (at most 64: splits >= 2), 4
+    // consecutive columns per pass, the CTA's blockDim / 64 threads of a row
+    // on every (blockDim / 64)-th column group.
     cluster_sync();
     const TileCoord c = tile_coord<BN>(g, blockIdx.x);
-    const int R = (BM + g.splits - 1) / g.splits;
+    const int splits = g.splits, gM = g.M, gN = g.N;
+    const long long ldo = g.ldo;
+    const int R = (BM + splits - 1) / splits;
     const int r0 = c.split * R, r1 = min(BM, r0 + R);
-    const int nrows = max(0, r1 - r0), ncols = min(c.bn, g.N - c.n0);
-    const int total = nrows * ((ncols + 3) / 4);
+    const int nrows = max(0, r1 - r0), ncols = min(c.bn, gN - c.n0);
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     const float* recv = reinterpret_cast<const float*>(epi_area + C::kStageArea);
     const bf16* pre = reinterpret_cast<const bf16*>(epi_area);
     const int ra = r0 & ~7;
-    // (compact loops: this code runs once per CTA, so its instructions are
-    // fetched cold; a short body costs less than an unrolled one)
-#pragma unroll 1
-    for (int e = threadIdx.x; e < total; e += blockDim.x) {
-      const int lr = e % nrows, lc = 4 * (e / nrows);
-      const int mm = c.m * BM + r0 + lr, nn = c.n0 + lc;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-      for (int sp = 0; sp < g.splits; ++sp) {
-        const float4 x = *reinterpret_cast<const float4*>(recv + (sp * R + lr) * C::kCsplitPitch + lc);
-        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
-      }
-      if (mm >= g.M) continue;
-      const float w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll 1
-      for (int k = 0; k < 4 && nn + k < g.N; ++k) {
-        const float a = has_aux ? __bfloat162float(pre[(lc + k) * C::kAuxPitch + r0 + lr - ra]) : 0.0f;
-        epi_store_one<KIND>(g, static_cast<long long>(nn + k) * g.ldo + mm, nn + k, w[k], a);
+    const int lr = threadIdx.x & 63, gstep = blockDim.x >> 6;
+    const int mm = c.m * BM + r0 + lr;
+    if (lr < nrows && mm < gM) {
+      for (int lc = 4 * (threadIdx.x >> 6); lc < ncols; lc += 4 * gstep) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < splits; ++sp) {
+          const float4 x = ld_shared_f4(recv + (sp * R + lr) * C::kCsplitPitch + lc);
+          v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+        }
+        const float w[4] = {v.x, v.y, v.z, v.w};
+        const int nn = c.n0 + lc;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (nn + k >= gN) break;
+          const float a = has_aux ? ld_shared_bf16(pre + (lc + k) * C::kAuxPitch + r0 + lr - ra) : 0.0f;
+          epi_store_one<KIND>(g, (nn + k) * ldo + mm, nn + k, w[k], a);
+        }
       }
     }
   } else if (!PAIR && g.csplit && g.splits > 1 && KIND != EPI_F32_PARTIAL && blockIdx.x < g.tiles) {

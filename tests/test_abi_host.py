@@ -135,8 +135,10 @@ def test_workspace_queries(lib):
             + r256(T * Di * 4) + r256(T // 2 * 64 * 4))
     assert abi.sambay_scan_prefill_workspace(d) == want
     # bf16 decode step: conv output, x_proj partials of 128 slices of 40
-    # channels, the split delta, B | C
-    step64 = r256(64 * Di * 4) + r256(128 * ldx * 64 * 4) + r256(2 * 64 * 160 * 2) + r256(64 * 32 * 4)
+    # channels, the split delta, B | C, and the single-kernel step's
+    # generation word + two meeting flags per slice (a 128-byte line each)
+    step64 = (r256(64 * Di * 4) + r256(128 * ldx * 64 * 4) + r256(2 * 64 * 160 * 2) + r256(64 * 32 * 4)
+              + r256(16 * (1 + 2 * 128) * 8))
     assert abi.sambay_scan_step_workspace(abi.make_dims(64, 999, 2560, 5120)) == step64
     assert step64 <= abi.NOALLOC_SCRATCH_BYTES
     # float32 decode step: conv output, x_proj output, dt and B | C pairs

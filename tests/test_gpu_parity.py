@@ -194,6 +194,27 @@ def test_decode_steps_equal_oracle_prefill(name):
     np.testing.assert_array_equal(host(cs), r["conv_state"])
 
 
+@pytest.mark.parametrize("B", [1, 5, 64, 65, 130])
+def test_decode_step_batches(B):
+    """bf16 decode steps at batches on both sides of 64 sequences (one kernel
+    over all slices up to 64; three kernels with sequence groups beyond):
+    every step's readout and the final state against the oracle's prefill
+    over the same tokens."""
+    d = synth.Dims(B, 12, 128, 256, 16, 4, 16, synth.BF16)
+    seed = 26 + B
+    w = synth.scan_weights(d, seed)
+    u = synth.scan_inputs(d, seed)
+    L0 = 8
+    layer = ScanLayer(w, d.d_model, abi.BF16)
+    _, h, cs = layer.prefill(to_device(u[:, :L0], abi.BF16))
+    r = ref.scan_prefill_ref(u, w)
+    for i in range(L0, d.seqlen):
+        m = layer.step(to_device(np.ascontiguousarray(u[:, i]), abi.BF16), h, cs)
+        assert_close(host(m), r["M"][:, i], TOL_BF16, f"B={B} step {i}")
+    assert_close(host(h), r["ssm_state"], TOL_BF16, f"B={B} state after steps")
+    np.testing.assert_array_equal(host(cs), r["conv_state"])
+
+
 def test_decode_state_save_restore_is_bit_identical():
     d = SMALL["bf16"]
     seed = 25
