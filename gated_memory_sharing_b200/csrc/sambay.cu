@@ -251,8 +251,9 @@ ScanWs scan_ws_layout(const sambay_dims* d, long long T, bool step = false) {
   w.xdbl = off;  off += round256(static_cast<size_t>(T * ldx) * 4);
   w.delta = off; off += tc ? round256(static_cast<size_t>(T) * 2 * rank_pad(static_cast<int>(R)) * 2) : 0;
   w.dt = off;    off += round256(static_cast<size_t>(T * Di) * 4);
-  // B | C regrouped into token pairs: ceil(L / 2) pairs of 64 floats per sequence
-  w.bcp = off;   off += round256(static_cast<size_t>(d->batch) * ((T / d->batch + 1) / 2) * 64 * 4);
+  // B | C regrouped into token pairs for the prefill scan: ceil(L / 2) pairs
+  // of 64 floats per sequence (the decode step reads xdbl instead)
+  w.bcp = off;   off += step ? 0 : round256(static_cast<size_t>(d->batch) * ((T / d->batch + 1) / 2) * 64 * 4);
   w.total = off;
   return w;
 }
@@ -643,11 +644,11 @@ sambay::simt::Args simt_args(const float* A, long long sam, long long sak, const
 // x_proj + dt_proj for `rows` tokens whose conv output is ws.uc:
 //   xdbl = uc W_x^T,  dt = softplus(delta W_dt^T + b_dt)
 sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
-                          long long rows, uint8_t* ws, const ScanWs& L, cudaStream_t st) {
+                          long long rows, uint8_t* ws, const ScanWs& L, cudaStream_t st, bool prefill) {
   const int Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
   float* xdbl = reinterpret_cast<float*>(ws + L.xdbl);
   float* dt = reinterpret_cast<float*>(ws + L.dt);
-  float* bcp = reinterpret_cast<float*>(ws + L.bcp);
+  float* bcp = prefill ? reinterpret_cast<float*>(ws + L.bcp) : nullptr;   // B | C segments: prefill only
   if (d->io == SAMBAY_BF16) {
     const bf16* uc = reinterpret_cast<const bf16*>(ws + L.uc);
     bf16* delta = reinterpret_cast<bf16*>(ws + L.delta);
@@ -692,7 +693,7 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
         simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
                   ldx, Di, xdbl, ldx),
         st));
-    {
+    if (prefill) {
       ProfScope ps_bc("bc_pairs", st);
       sambay::scan::bc_pairs_kernel<<<grid_for(rows * 2 * d->d_state, 256, 1 << 20), 256, 0, st>>>(
           xdbl, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, ldx);
@@ -774,7 +775,7 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
-  SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st));
+  SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st, true));
   {
     sambay::scan::ScanParams<T> p{};
     p.uc = uc;
@@ -895,7 +896,7 @@ sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, con
     const StepPlan sp = step_plan(d);
     if (sp.ok) return scan_step_fused(dev, sms, w, d, sp, u_t, m_t, ssm_state, conv_state, ws, st);
   }
-  const ScanWs L = scan_ws_layout(d, B);
+  const ScanWs L = scan_ws_layout(d, B, true);
   T* uc = reinterpret_cast<T*>(ws + L.uc);
   constexpr int VEC = 16 / sizeof(T);
   auto sc = sambay::scan::step_conv_kernel<T>;
@@ -909,7 +910,7 @@ sambay_status scan_step_impl(int dev, int sms, const sambay_scan_weights* w, con
       static_cast<const T*>(w->conv_b), uc, d->batch, d->d_inner);
   }
   if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
-  SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st));
+  SAMBAY_TRY(projections(dev, sms, w, d, B, ws, L, st, false));
   ProfScope ps("step_scan", st);
   const cudaError_t e = launch_k(ss, dim3(grid_for(B * d->d_inner * 4, 256, 1 << 20)), dim3(256), 0, st, true, 1,
                                  static_cast<const T*>(uc), reinterpret_cast<const float*>(ws + L.dt),

@@ -250,7 +250,7 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
       reinterpret_cast<__nv_bfloat162*>(dh)[1] = __halves2bfloat162(hi[2], hi[3]);
       reinterpret_cast<__nv_bfloat162*>(dl)[0] = __halves2bfloat162(lo[0], lo[1]);
       reinterpret_cast<__nv_bfloat162*>(dl)[1] = __halves2bfloat162(lo[2], lo[3]);
-    } else {
+    } else if (bcp != nullptr) {
       // B | C columns, also regrouped into token pairs for the prefill scan
       const float a[4] = {acc.x, acc.y, acc.z, acc.w};
       const int rr = static_cast<int>(row), b = rr / L, t = rr % L, Lh = (L + 1) >> 1;
