@@ -209,17 +209,19 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
     const bool valid = i < total4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (valid) {
-      // a batch of this lane's splits loaded together, then added in order
+      // a batch of this lane's splits loaded together (with one lane per
+      // group, all of them: fewer than 16 splits), then added in order
+      constexpr int kBatch = LPG == 1 ? 16 : 4;
 #pragma unroll 1
-      for (int s0 = sub; s0 < splits; s0 += 4 * LPG) {
-        float4 p[4];
+      for (int s0 = sub; s0 < splits; s0 += kBatch * LPG) {
+        float4 p[kBatch];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
           const int sp = s0 + j * LPG;
           p[j] = ldcg_or_zero(partials + (sp < splits ? sp * split_stride + 4 * i : 0), sp < splits);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
           acc.x += p[j].x; acc.y += p[j].y; acc.z += p[j].z; acc.w += p[j].w;
         }
       }

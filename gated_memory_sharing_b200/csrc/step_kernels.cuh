@@ -443,9 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1) step_scan_kernel(const StepParams
 // cooperatively, so all CTAs are resident together, and the two points where
 // the step needs every slice's result (the x_proj sum over channels, then its
 // use by every slice) are grid-wide meeting points instead of kernel
-// boundaries.  The slice's state arrives as one tensor copy and its W_dt, A,
-// b_dt and D slices by cp.async, both issued behind the conv's own loads and
-// landing under the conv, the partial x_proj and both meetings.
+// boundaries.  The slice's W_dt, A, b_dt and D slices arrive by cp.async
+// behind the conv's own loads, and its state as one tensor copy issued once
+// the conv is done; both land under the partial x_proj and the meetings.
 //
 //   phase 0   conv of the slice (uc stays in shared memory), partial x_proj
 //             sums part[slice][seq][j] (m16n8k16)
@@ -667,14 +667,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) step_fused_kernel(const Step
     }
   }
 
-  // ---- phase 0b, behind those loads: the slice's state as ONE tensor copy
-  // (box {128 floats, chan / 8, B} of h viewed as [B][Di / 8][128]) landing
-  // on `mb`, and the W_dt rows, A, b_dt and D slices (cp.async); all of it
-  // lands while the conv, the x_proj and both meetings run
-  if (tid == 0) {
-    mb_expect_tx(mb, static_cast<uint32_t>(B) * chan * kStateN * 4);
-    tma_load_3d(h_s, &hmap, mb, 0, c0 / 8, 0);
-  }
+  // ---- phase 0b, behind those loads: the W_dt rows, A, b_dt and D slices
+  // (cp.async), landing while the conv, the x_proj and both meetings run.
+  // The slice's state follows after the conv as ONE tensor copy (box {128
+  // floats, chan / 8, B} of h viewed as [B][Di / 8][128]) landing on `mb`.
   {
     const int rc = R / 8;
     for (int i = tid; i < chan * rc; i += kFusedThreads) {
@@ -732,6 +728,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) step_fused_kernel(const Step
     ucs[r * kUcsPitch + c] = __float2bfloat16_rn(0.0f);
   }
   __syncthreads();
+  // the slice's state, once the conv's own reads are done (so they did not
+  // queue behind it); it lands under the x_proj and both meetings
+  if (tid == 0) {
+    mb_expect_tx(mb, static_cast<uint32_t>(B) * chan * kStateN * 4);
+    tma_load_3d(h_s, &hmap, mb, 0, c0 / 8, 0);
+  }
 
   // ---- phase 0d: partial x_proj D[j][n] = sum_{c in slice} W_x[j][c] ucs[n][c],
   // stored as part[slice][seq][j]
