@@ -579,16 +579,18 @@ def bench_decode(args, ctx, name):
 
     # ---- the stated horizon back to back (graphs of 64 steps, no flush)
     horizon = synth.DECODE_STEPS["decode_b64" if name == "decode_b64" else "sharing_b2_l8192"]
-    hz = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    barrier(world)
-    torch.cuda.synchronize()
-    hz[0].record(stream)
-    for _ in range(horizon // 64):
-        g64.replay()
-    hz[1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    horizon_ms = max_over_ranks(hz[0].elapsed_time(hz[1]), world, device)
+    horizon_ms = None
+    if not args.no_horizon:
+        hz = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        barrier(world)
+        torch.cuda.synchronize()
+        hz[0].record(stream)
+        for _ in range(horizon // 64):
+            g64.replay()
+        hz[1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        horizon_ms = max_over_ranks(hz[0].elapsed_time(hz[1]), world, device)
 
     # ---- per-kernel breakdown of single steps (L2 flushed before each)
     per_kernel = {}
@@ -634,7 +636,8 @@ def bench_decode(args, ctx, name):
         "config": config_of(name, d, layers, True),
         "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the step events)",
         "prompt_prefill_ms": prompt_ms,
-        "horizon": {"steps": horizon, "ms": horizon_ms, "us_per_step": 1e3 * horizon_ms / horizon,
+        "horizon": None if horizon_ms is None else
+                   {"steps": horizon, "ms": horizon_ms, "us_per_step": 1e3 * horizon_ms / horizon,
                     "note": "back-to-back steps in graphs of 64, L2 not flushed"},
         "kernels_us": kernels_us,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -794,6 +797,8 @@ def main():
     ap.add_argument("--workload", choices=WORKLOADS, default=HEADLINE)
     ap.add_argument("--only-headline", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-horizon", action="store_true",
+                    help="decode workloads: skip the back-to-back run over the stated horizon (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

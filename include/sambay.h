@@ -141,13 +141,22 @@ SAMBAY_API sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const
  * sambay_scan_step - one decode token per sequence: the prefill with L = 1
  * on the carried state, updating ssm_state and conv_state IN PLACE [GMU]
  * (constant-size state), [MAMBA].  dims->seqlen is ignored.  In SAMBAY_BF16
- * mode this is three kernels over channel slices (about one slice of up to
- * 48 channels per SM): conv + the slice's partial x_proj sums; their sum in a
- * fixed slice order; dt_proj + the state update, whose state and weight
- * slices are copied before it waits for the other two.  ws holds the conv
- * output, the partial sums, delta and B | C:
- *   B * (4 Di + 4 ceil(Di / chan) (R + 2N) + 4 R16 + 8 N) bytes (R16 = R
- *   rounded up to 16), about 7.7 MB for 64 sequences at d_inner 5120.
+ * mode the work is cut into channel slices (about one slice of up to 48
+ * channels per SM).  Up to 64 sequences it is ONE cooperative kernel, one CTA
+ * per slice, all resident at once: conv + the slice's partial x_proj sums,
+ * a grid-wide meeting point, each CTA's share of the sums over slices (a
+ * fixed order), a second meeting point, dt_proj + the state update; the
+ * slice's state arrives by one tensor copy issued after the conv.  Above 64
+ * sequences (or where the slices do not fit the GPU at one CTA per SM) it is
+ * three kernels with the same stages, chained.  ws holds the conv output,
+ * the partial sums, delta, B | C and the meeting points' words (a
+ * generation word and two flags per slice, 128 bytes each; any contents are
+ * accepted, and a call leaves them consistent for the next):
+ *   B * (4 Di + 4 ceil(Di / chan) (R + 2N) + 4 R16 + 8 N) bytes + 128 *
+ *   (1 + 2 ceil(Di / chan)) (R16 = R rounded up to 16), about 7.7 MB for 64
+ *   sequences at d_inner 5120.  Calls that share a ws must not overlap on
+ *   the GPU (the meeting words are per ws).  After a SAMBAY_ERR_TIMEOUT the
+ *   ws's meeting words may be inconsistent: zero the ws before reusing it.
  * SAMBAY_F32 runs a chain of float32 kernels that exchange their
  * intermediates through ws.
  *
@@ -327,7 +336,10 @@ SAMBAY_API sambay_status sambay_cross_attn_decode(const sambay_attn_dims* dims, 
  *
  *   - The scratch it needs is what sambay_scan_step_workspace(dims) reports
  *     (see sambay_scan_step): about 7.7 MB for 64 bf16 sequences at d_inner
- *     5120, and for SAMBAY_F32 about B * (2 * Di + R + 2N + 64) * 4 bytes.
+ *     5120, and for SAMBAY_F32 about B * (2 * Di + R + 2N) * 4 bytes.
+ *     The bf16 step's meeting words (see sambay_scan_step) live in that
+ *     array too; after a SAMBAY_ERR_TIMEOUT from this entry point they may
+ *     be inconsistent until the process restarts.
  *     Sizes whose sambay_scan_step_workspace(dims) exceeds
  *     SAMBAY_NOALLOC_SCRATCH_BYTES are rejected with SAMBAY_ERR_UNSUPPORTED
  *     before any launch; check that query against the limit before relying
