@@ -22,6 +22,11 @@ Sources (cited per function in :mod:`oracle.sambay_ref`):
   input-dependent Δ/B/C projections, softplus Δ, Ā = exp(ΔA), B̄ = ΔB,
   the recurrence and its readout.  Used as mathematics only.
 
+* Mamba-2's SSD layer (Dao & Gu 2024, "Transformers are SSMs"), for the
+  SambaY-2 ablation row (Paper-Notes page, 实验关键数据 > 消融实验): one
+  scalar decay per head, B and C shared by the heads; in
+  :mod:`oracle.ssd_ref`.  Used as mathematics only.
+
 Parity status per function: every function is pinned by a CPU test in
 ``tests/test_oracle_pins.py`` against something other than itself (closed
 forms, brute force, library routines, hand-derived golden values).  The one
@@ -47,4 +52,11 @@ from .sambay_ref import (  # noqa: F401
     mlp_representation_ref,
     sambay_mlp_gmu_ref,
     cross_attention_decode_ref,
+)
+from .ssd_ref import (  # noqa: F401
+    ssd_recurrent,
+    ssd_chunked,
+    ssd_matrix,
+    mamba2_scan_ref,
+    mamba2_step_ref,
 )
