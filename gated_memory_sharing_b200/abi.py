@@ -46,6 +46,8 @@ EXPORTS = (
     "sambay_decode_step",
     "sambay_cross_attn_decode_workspace",
     "sambay_cross_attn_decode",
+    "sambay_ssd_prefill_workspace",
+    "sambay_ssd_prefill",
     "sambay_gmu_step_stall_test",
     "sambay_profile_begin",
     "sambay_profile_end",
@@ -96,6 +98,29 @@ class AttnDims(ctypes.Structure):
     ]
 
 
+class SsdDims(ctypes.Structure):
+    """sambay_ssd_dims: the SambaY-2 (Mamba-2) layer's sizes."""
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("seqlen", ctypes.c_int32),
+        ("nheads", ctypes.c_int32),
+        ("headdim", ctypes.c_int32),
+        ("d_state", ctypes.c_int32),
+        ("d_conv", ctypes.c_int32),
+        ("io", ctypes.c_int32),
+    ]
+
+
+class SsdWeights(ctypes.Structure):
+    _fields_ = [
+        ("conv_w", ctypes.c_void_p),
+        ("conv_b", ctypes.c_void_p),
+        ("dt_bias", ctypes.c_void_p),
+        ("A", ctypes.c_void_p),
+        ("D", ctypes.c_void_p),
+    ]
+
+
 class GmuWeights(ctypes.Structure):
     _fields_ = [
         ("W1", ctypes.c_void_p),
@@ -120,6 +145,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     pd, pw = ctypes.POINTER(Dims), ctypes.POINTER(ScanWeights)
     pg = ctypes.POINTER(GmuWeights)
     pa = ctypes.POINTER(AttnDims)
+    psd, psw = ctypes.POINTER(SsdDims), ctypes.POINTER(SsdWeights)
     sig = {
         "sambay_scan_prefill_workspace": (sz, [pd]),
         "sambay_scan_step_workspace": (sz, [pd]),
@@ -137,6 +163,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sambay_decode_step_workspace": (sz, [pd, i32]),
         "sambay_cross_attn_decode_workspace": (sz, [pa]),
         "sambay_cross_attn_decode": (ctypes.c_int, [pa, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp]),
+        "sambay_ssd_prefill_workspace": (sz, [psd]),
+        "sambay_ssd_prefill": (ctypes.c_int, [psw, psd, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
         "sambay_decode_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, i32, pg, vp, vp, sz, vp]),
         "sambay_gmu_step_stall_test": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz,
                                                       ctypes.c_uint64, vp]),
@@ -243,6 +271,18 @@ def sambay_cross_attn_decode(dims: AttnDims, q, K, V, out, scale: float, ws, str
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("sambay_cross_attn_decode", load().sambay_cross_attn_decode(
         ctypes.byref(dims), _p(q), _p(K), _p(V), _p(out), scale, _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_ssd_prefill_workspace(dims: SsdDims) -> int:
+    return load().sambay_ssd_prefill_workspace(ctypes.byref(dims))
+
+
+def sambay_ssd_prefill(w: SsdWeights, dims: SsdDims, xbc, dt_raw, M, ssm_state, conv_state, zero_init: bool, ws,
+                       stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_ssd_prefill", load().sambay_ssd_prefill(
+        ctypes.byref(w), ctypes.byref(dims), _p(xbc), _p(dt_raw), _p(M), _p(ssm_state), _p(conv_state),
+        1 if zero_init else 0, _p(ws), ws_bytes, _stream(stream)))
 
 
 def sambay_decode_step_workspace(dims: Dims, n_layers: int) -> int:

@@ -17,6 +17,7 @@
 #include "attn_kernels.cuh"
 #include "scan_kernels.cuh"
 #include "simt_gemm.cuh"
+#include "ssd_kernels.cuh"
 #include "step_kernels.cuh"
 #include "tc_gemm.cuh"
 
@@ -1414,6 +1415,106 @@ sambay_status sambay_cross_attn_decode(const sambay_attn_dims* a, const void* q,
   p.scale_log2 = sc * 1.4426950408889634f;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return a->head_dim == 64 ? attn_launch<64>(dev, sms, p, st) : attn_launch<128>(dev, sms, p, st);
+}
+
+// ------------------------------------------------------------ SambaY-2 (Mamba-2 SSD)
+
+namespace {
+
+sambay_status ssd_check(const sambay_ssd_dims* d) {
+  if (!d) return SAMBAY_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->seqlen <= 0 || d->nheads <= 0 || d->headdim <= 0 || d->d_state <= 0 ||
+      d->d_conv <= 0)
+    return SAMBAY_ERR_INVALID_ARG;
+  if (d->io != SAMBAY_BF16 && d->io != SAMBAY_F32) return SAMBAY_ERR_INVALID_ARG;
+  if (d->io != SAMBAY_BF16 || d->headdim != sambay::ssd::kP || (d->d_state != 64 && d->d_state != 128) ||
+      d->d_conv != 4)
+    return SAMBAY_ERR_UNSUPPORTED;
+  const long long C = static_cast<long long>(d->nheads) * d->headdim + 2LL * d->d_state;
+  if (C % 32 != 0 || C > (1LL << 24) || static_cast<long long>(d->batch) * d->seqlen > (1LL << 26))
+    return SAMBAY_ERR_UNSUPPORTED;
+  return SAMBAY_OK;
+}
+
+}  // namespace
+
+size_t sambay_ssd_prefill_workspace(const sambay_ssd_dims* d) {
+  if (ssd_check(d) != SAMBAY_OK) return 0;
+  const size_t C = static_cast<size_t>(d->nheads) * d->headdim + 2 * static_cast<size_t>(d->d_state);
+  return round256(static_cast<size_t>(d->batch) * d->seqlen * C * 4);
+}
+
+sambay_status sambay_ssd_prefill(const sambay_ssd_weights* w, const sambay_ssd_dims* d, const void* xbc,
+                                 const void* dt_raw, void* M, float* ssm_state, void* conv_state, int32_t zero_init,
+                                 void* ws, size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(ssd_check(d));
+  if (!w) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({w->conv_w, w->conv_b, w->dt_bias, w->A, w->D}));
+  SAMBAY_TRY(check_ptrs({xbc, dt_raw, M, ssm_state, conv_state}));
+  if (M == xbc) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_ssd_prefill_workspace(d)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int C = d->nheads * d->headdim + 2 * d->d_state;
+  bf16* xc = static_cast<bf16*>(ws);
+  {
+    sambay::scan::ConvParams<bf16> p{static_cast<const bf16*>(xbc), static_cast<const bf16*>(conv_state),
+                                     static_cast<const bf16*>(w->conv_w), static_cast<const bf16*>(w->conv_b), xc,
+                                     d->batch, d->seqlen, C, zero_init ? 1 : 0};
+    using sambay::scan::kConvTT;
+    auto c64 = sambay::scan::conv_silu_kernel<bf16, 64>;
+    auto c32 = sambay::scan::conv_silu_kernel<bf16, 32>;
+    SAMBAY_MAX_CARVEOUT(c64, dev);
+    SAMBAY_MAX_CARVEOUT(c32, dev);
+    ProfScope ps("ssd_conv_silu", st);
+    if (C % 64 == 0) {
+      dim3 grid(C / 64, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
+      c64<<<grid, 64 / 4 * (kConvTT / 4), 0, st>>>(p);
+    } else {
+      dim3 grid(C / 32, (d->seqlen + kConvTT - 1) / kConvTT, d->batch);
+      c32<<<grid, 32 / 4 * (kConvTT / 4), 0, st>>>(p);
+    }
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+  }
+  {
+    auto kern = sambay::ssd::ssd_chunk_scan_kernel;
+    static bool attr_set[kMaxDevices] = {};
+    const sambay::ssd::SsdLayout ly(d->d_state);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sambay::ssd::SsdLayout(sambay::ssd::kMaxN).bytes) != cudaSuccess)
+        return SAMBAY_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+    sambay::ssd::SsdParams p{};
+    p.xc = xc;
+    p.dt_raw = static_cast<const bf16*>(dt_raw);
+    p.dt_bias = w->dt_bias;
+    p.A = w->A;
+    p.D = w->D;
+    p.h = ssm_state;
+    p.M = static_cast<bf16*>(M);
+    p.Bt = d->batch;
+    p.L = d->seqlen;
+    p.H = d->nheads;
+    p.N = d->d_state;
+    p.zero_init = zero_init ? 1 : 0;
+    ProfScope ps("ssd_chunk_scan", st);
+    if (launch_k(kern, dim3(d->nheads, d->batch), dim3(sambay::ssd::kThreads), ly.bytes, st, true, 1, p) !=
+        cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+  }
+  {
+    // after the conv has read the old window
+    const long long n = static_cast<long long>(d->batch) * C;
+    ProfScope ps("ssd_conv_state", st);
+    if (launch_k(sambay::ssd::conv_state_update_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
+                 st, true, 1, static_cast<const bf16*>(xbc), static_cast<bf16*>(conv_state), d->batch, d->seqlen, C,
+                 zero_init ? 1 : 0) != cudaSuccess)
+      return SAMBAY_ERR_CUDA;
+  }
+  return SAMBAY_OK;
 }
 
 sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const sambay_dims* d,

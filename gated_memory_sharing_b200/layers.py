@@ -227,3 +227,51 @@ class MLPMemory:
             self._ws[rows] = ws
         abi.sambay_mlp_memory(d, rows, X, self.W_g, self.W_u, M, ws, stream)
         return M
+
+
+class Mamba2Scan:
+    """The SambaY-2 memory: a Mamba-2 (SSD) layer's readout over a prompt."""
+
+    def __init__(self, w: dict, io: int = abi.BF16, device="cuda"):
+        self.io = io
+        self.dtype = io_dtype(io)
+        self.nheads = int(w["A"].shape[0])
+        self.headdim = int(w["P"])
+        self.d_state = int(w["N"])
+        self.channels, self.d_conv = w["conv_w"].shape
+        self.conv_w = to_device(w["conv_w"], io, device)
+        self.conv_b = to_device(w["conv_b"], io, device)
+        self.dt_bias = to_device_f32(w["dt_bias"], device)
+        self.A = to_device_f32(w["A"], device)
+        self.D = to_device_f32(w["D"], device)
+        self.abi_w = abi.SsdWeights(self.conv_w.data_ptr(), self.conv_b.data_ptr(), self.dt_bias.data_ptr(),
+                                    self.A.data_ptr(), self.D.data_ptr())
+        self.device = device
+        self._ws = {}
+
+    def dims(self, batch: int, seqlen: int) -> abi.SsdDims:
+        return abi.SsdDims(batch, seqlen, self.nheads, self.headdim, self.d_state, self.d_conv, self.io)
+
+    def new_state(self, batch: int):
+        h = torch.zeros(batch, self.nheads, self.headdim, self.d_state, dtype=torch.float32, device=self.device)
+        cs = torch.zeros(batch, self.channels, self.d_conv, dtype=self.dtype, device=self.device)
+        return h, cs
+
+    def prefill(self, xbc, dt_raw, ssm_state=None, conv_state=None, M=None, fresh=None, stream=None):
+        """xbc [B, L, C], dt_raw [B, L, H] -> M [B, L, H * P]; states as for
+        ScanLayer.prefill (returned, updated in place)."""
+        B, L, _ = xbc.shape
+        if fresh is None:
+            fresh = ssm_state is None
+        if ssm_state is None:
+            ssm_state, conv_state = self.new_state(B)
+        if M is None:
+            M = torch.empty(B, L, self.nheads * self.headdim, dtype=self.dtype, device=self.device)
+        d = self.dims(B, L)
+        n = abi.sambay_ssd_prefill_workspace(d)
+        ws = self._ws.get((B, L))
+        if ws is None:
+            ws = workspace(n, self.device)
+            self._ws[(B, L)] = ws
+        abi.sambay_ssd_prefill(self.abi_w, d, xbc, dt_raw, M, ssm_state, conv_state, fresh, ws, stream)
+        return M, ssm_state, conv_state

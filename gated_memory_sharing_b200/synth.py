@@ -180,6 +180,56 @@ def attention_inputs(batch: int, kv_len: int, q_heads: int, kv_heads: int, head_
             round_bf16(r.normal("V", (batch, kv_len, kv_heads, head_dim))))
 
 
+@dataclasses.dataclass(frozen=True)
+class SsdDims:
+    """The SambaY-2 (Mamba-2) layer: d_inner = nheads * headdim, one group of
+    B and C (d_state each), conv over C = d_inner + 2 d_state channels."""
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int = 64
+    d_state: int = 128
+    d_conv: int = 4
+    io: str = BF16
+
+    @property
+    def channels(self) -> int:
+        return self.nheads * self.headdim + 2 * self.d_state
+
+
+# The SambaY-2 variant of the prefill workload: d_inner 5120 as 80 heads of 64,
+# d_state 128 (Mamba-2's defaults; the pages give no sizes for the variant).
+SSD_WORKLOAD = SsdDims(1, 2048, 80, 64, 128, 4, BF16)
+SSD_WORKLOAD_SEED = 1000 + 17
+
+
+def ssd_weights(d: SsdDims, seed: int) -> dict:
+    """Mamba-2 layer parameters for the readout: conv over [x | B | C], dt bias
+    with softplus(dt_bias) in [1e-3, 1e-1], A = -exp(U[log 1, log 16]) per head,
+    D ~ U(0.5, 1.5) per head (the Mamba-1 recipe per head)."""
+    r = Draws(seed)
+    C, H, K = d.channels, d.nheads, d.d_conv
+    dt0 = np.exp(r.uniform("ssd_dt0", (H,), np.log(1e-3), np.log(1e-1)))
+    return dict(
+        conv_w=to_io(r.normal("ssd_conv_w", (C, K), 1.0 / np.sqrt(K)), d.io),
+        conv_b=to_io(r.uniform("ssd_conv_b", (C,), -1.0 / np.sqrt(K), 1.0 / np.sqrt(K)), d.io),
+        dt_bias=(dt0 + np.log(-np.expm1(-dt0))).astype(np.float32),
+        A=(-np.exp(r.uniform("ssd_A", (H,), np.log(1.0), np.log(16.0)))).astype(np.float32),
+        D=r.uniform("ssd_D", (H,), 0.5, 1.5).astype(np.float32),
+        P=d.headdim,
+        N=d.d_state,
+    )
+
+
+def ssd_inputs(d: SsdDims, seed: int, seqlen=None):
+    """(xbc [Bt, L, C], dt_raw [Bt, L, H]): the in_proj slices, N(0, 1) and
+    N(0, 0.5^2) (dt_raw around the bias), I/O-rounded."""
+    r = Draws(seed)
+    L = d.seqlen if seqlen is None else seqlen
+    return (to_io(r.normal("xbc", (d.batch, L, d.channels)), d.io),
+            to_io(r.normal("dt_raw", (d.batch, L, d.nheads), 0.5), d.io))
+
+
 def workload(name: str):
     """(dims, default seed) of a named workload."""
     return WORKLOADS[name], 1000 + WORKLOAD_IDS[name]

@@ -320,6 +320,59 @@ SAMBAY_API sambay_status sambay_cross_attn_decode(const sambay_attn_dims* dims, 
                                                   const void* K, const void* V, void* out, float scale,
                                                   void* ws, size_t ws_bytes, sambay_stream_t stream);
 
+/* ---------------------------------------------------------------------- */
+/* SambaY-2: the memory readout of a Mamba-2 (SSD) layer                    */
+/* ---------------------------------------------------------------------- */
+
+/* Sizes of the Mamba-2 layer whose readout is M in the SambaY-2 variant
+ * ("Decoder-Hybrid-Decoder Architecture ...", Paper-Notes page, 实验关键数据 >
+ * 消融实验, row SambaY-2: Mamba replaced by Mamba-2, a scalar forget gate per
+ * head).  One group: B and C are shared by all heads. */
+typedef struct {
+  int32_t batch;     /* Bt sequences                                        */
+  int32_t seqlen;    /* L tokens                                            */
+  int32_t nheads;    /* H heads; d_inner = H * headdim                       */
+  int32_t headdim;   /* P: 64                                               */
+  int32_t d_state;   /* N: 64 or 128                                        */
+  int32_t d_conv;    /* K: 4                                                */
+  int32_t io;        /* sambay_dtype: SAMBAY_BF16                           */
+} sambay_ssd_dims;
+
+/* Device pointers.  C = H * P + 2 N conv channels ([x | B | C]). */
+typedef struct {
+  const void* conv_w;    /* [C, K] io   depthwise causal conv taps (tap K-1 on
+                            the current token)                              */
+  const void* conv_b;    /* [C]    io                                       */
+  const float* dt_bias;  /* [H]    f32  dt = softplus(dt_raw + dt_bias)      */
+  const float* A;        /* [H]    f32  negative; decay exp(dt A) per head   */
+  const float* D;        /* [H]    f32  skip weight                         */
+} sambay_ssd_weights;
+
+/*
+ * sambay_ssd_prefill - the SambaY-2 memory M of a prompt: the causal conv +
+ * SiLU of the in_proj slice [x | B | C], dt = softplus(dt_raw + dt_bias), and
+ * the SSD recurrence of Mamba-2 (Dao & Gu 2024, "Transformers are SSMs"):
+ *     H_t = exp(dt_t A_h) H_{t-1} + dt_t x_t B_t^T,   y_t = H_t C_t + D_h x_t
+ * per head h (x_t, y_t in R^P, H in R^{P x N}), M = y.  Computed chunk by
+ * chunk (64 tokens) on the tensor cores: per chunk and head the products
+ * C B^T, (masked, decay-scaled) W X, C H and (B scaled)^T X, with the fp32
+ * state carried across chunks; operands bf16, accumulation fp32.
+ *
+ *   xbc [Bt, L, C] io in;  dt_raw [Bt, L, H] io in;  M [Bt, L, H*P] io out;
+ *   ssm_state [Bt, H, P, N] f32 in/out (read unless zero_init);
+ *   conv_state [Bt, C, K] io in/out (the left context unless zero_init; the
+ *   last K inputs on return).  io must be SAMBAY_BF16, P = 64, N in {64,
+ *   128}, K = 4, C a multiple of 32; other sizes return
+ *   SAMBAY_ERR_UNSUPPORTED.  M must not alias xbc.
+ *   ws: >= sambay_ssd_prefill_workspace(dims): the conv output as a bf16
+ *   split pair, Bt * L * C * 4 bytes.
+ */
+SAMBAY_API size_t sambay_ssd_prefill_workspace(const sambay_ssd_dims* dims);
+SAMBAY_API sambay_status sambay_ssd_prefill(const sambay_ssd_weights* w, const sambay_ssd_dims* dims,
+                                            const void* xbc, const void* dt_raw, void* M, float* ssm_state,
+                                            void* conv_state, int32_t zero_init, void* ws, size_t ws_bytes,
+                                            sambay_stream_t stream);
+
 /*
  * sambay_scan_step_noalloc - sambay_scan_step for callers that cannot
  * allocate device memory.  The paper has no counterpart; this is a property

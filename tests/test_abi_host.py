@@ -280,3 +280,28 @@ def test_product_path_has_no_oracle_or_fallback():
             abi.load("/nonexistent/libsambay.so")
         finally:
             abi._lib = abi._lib_backup
+
+
+def test_ssd_argument_errors(lib):
+    ok = abi.SsdDims(1, 2048, 80, 64, 128, 4, abi.BF16)
+    # the conv output as a bf16 split pair: L x (H P + 2 N) x 4 bytes
+    assert abi.sambay_ssd_prefill_workspace(ok) == 2048 * (80 * 64 + 256) * 4
+    p = _FakePtr(0x10000)
+    w = abi.SsdWeights(0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
+    for bad, code in ((abi.SsdDims(1, 64, 2, 64, 128, 4, abi.F32), 2),      # float32 I/O
+                      (abi.SsdDims(1, 64, 2, 128, 128, 4, abi.BF16), 2),    # head dim
+                      (abi.SsdDims(1, 64, 2, 64, 96, 4, abi.BF16), 2),      # d_state
+                      (abi.SsdDims(1, 64, 2, 64, 64, 3, abi.BF16), 2),      # conv width
+                      (abi.SsdDims(0, 64, 2, 64, 64, 4, abi.BF16), 1)):
+        assert abi.sambay_ssd_prefill_workspace(bad) == 0
+        with pytest.raises(abi.SambayError) as e:
+            abi.sambay_ssd_prefill(w, bad, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                                   _FakePtr(0x50000), True, p, 0)
+        assert e.value.code == code
+    with pytest.raises(abi.SambayError) as e:     # M aliases xbc
+        abi.sambay_ssd_prefill(w, ok, p, _FakePtr(0x20000), p, _FakePtr(0x40000), _FakePtr(0x50000), True, p, 0)
+    assert e.value.code == 1
+    with pytest.raises(abi.SambayError) as e:     # workspace too small
+        abi.sambay_ssd_prefill(w, ok, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
+                               _FakePtr(0x50000), True, p, 0)
+    assert e.value.code == 3
