@@ -1478,12 +1478,14 @@ sambay_status sambay_ssd_prefill(const sambay_ssd_weights* w, const sambay_ssd_d
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
   {
-    auto kern = sambay::ssd::ssd_chunk_scan_kernel;
+    auto kern = d->d_state == 128 ? sambay::ssd::ssd_chunk_scan_kernel<128> : sambay::ssd::ssd_chunk_scan_kernel<64>;
     static bool attr_set[kMaxDevices] = {};
     const sambay::ssd::SsdLayout ly(d->d_state);
     if (!attr_set[dev]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               sambay::ssd::SsdLayout(sambay::ssd::kMaxN).bytes) != cudaSuccess)
+      if (cudaFuncSetAttribute(sambay::ssd::ssd_chunk_scan_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sambay::ssd::SsdLayout(128).bytes) != cudaSuccess ||
+          cudaFuncSetAttribute(sambay::ssd::ssd_chunk_scan_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sambay::ssd::SsdLayout(64).bytes) != cudaSuccess)
         return SAMBAY_ERR_CUDA;
       attr_set[dev] = true;
     }

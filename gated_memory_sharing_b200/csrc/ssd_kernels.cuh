@@ -19,11 +19,13 @@
 // with W = G masked and scaled (64 x P, K = 64), C H_in (64 x P, K = N) and
 // S = (B scaled)^T X (N x P, K = 64).
 //
-// CTA: one (sequence, head), 4 warps, the chunks in order.  Warp w owns the
-// output rows t in [16 w, 16 w + 16) of the chunk and the state rows n in
-// [N w / 4, N (w + 1) / 4); the fp32 state lives in its MMA accumulator
-// registers across chunks, with a bf16 copy in shared memory for the carry
-// product.  Operands come from shared memory by ldmatrix (.trans where the
+// CTA: one (sequence, head), 8 warps, the chunks in order (chunk ck + 1's
+// tiles load while ck computes).  Warp w computes C B^T and W for the rows
+// t in [16 (w % 4), +16) and the s half w / 4, writes W to shared memory,
+// then the output rows t for the p half w / 4 (carry and W X); the state
+// rows n in [16 (w % (N / 16)), +16) (all P, or a P half when N = 64) live in
+// its MMA accumulator registers across chunks in fp32, with a bf16 copy in
+// shared memory for the carry product.  Operands come from shared memory by ldmatrix (.trans where the
 // stored tile is K-major for the operand); W goes from accumulator fragments
 // straight into A fragments.  Operands are bf16 (x, B, C: the hi half of the
 // conv output's split pair; W and the state copy rounded), accumulation and
@@ -37,7 +39,8 @@ namespace ssd {
 
 constexpr int kQ = 64;          // tokens per chunk
 constexpr int kP = 64;          // head dim
-constexpr int kThreads = 128;   // 4 warps
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxN = 128;      // d_state
 
 struct SsdParams {
@@ -57,17 +60,22 @@ struct SsdParams {
 constexpr int kPitchP = kP + 8;          // x tiles, state copy
 __host__ __device__ constexpr int pitch_n(int N) { return N + 8; }
 
+// Two buffers of the chunk tiles (x hi, x lo, B, C, dt, c): chunk ck + 1
+// loads while chunk ck computes.
 struct SsdLayout {
-  int x, xl, b, c, hs, dt, cs, bytes;
+  int x, xl, b, c, dt, cs, buf, hs, w, wr, bytes;
   __host__ __device__ SsdLayout(int N) {
     x = 0;                                   // bf16 [kQ][kPitchP]  x hi
     xl = x + kQ * kPitchP * 2;               // bf16 [kQ][kPitchP]  x lo
     b = xl + kQ * kPitchP * 2;               // bf16 [kQ][pitch_n]  B, then B scaled
     c = b + kQ * pitch_n(N) * 2;             // bf16 [kQ][pitch_n]  C
-    hs = c + kQ * pitch_n(N) * 2;            // bf16 [N][kPitchP]   state copy
-    dt = hs + N * kPitchP * 2;               // f32 [kQ]
+    dt = c + kQ * pitch_n(N) * 2;            // f32 [kQ]
     cs = dt + kQ * 4;                        // f32 [kQ] c_t log2(e)
-    bytes = cs + kQ * 4;
+    buf = cs + kQ * 4;                       // bytes of one buffer
+    hs = 2 * buf;                            // bf16 [N][kPitchP]   state copy
+    w = hs + N * kPitchP * 2;                // bf16 [kQ][kPitchP]  W (rows t, columns s)
+    wr = w + kQ * kPitchP * 2;               // f32 [kQ] state weights exp(c_end - c_s) dt_s
+    bytes = wr + kQ * 4;
   }
 };
 
@@ -121,183 +129,207 @@ __device__ __forceinline__ void frag_b_t(uint32_t (&b)[4], const bf16* tile, int
   ldsm_x4_t(b, tile + (k0 + (j & 1) * 8 + i) * pitch + n0 + (j >> 1) * 8);
 }
 
+template <int N>
 __global__ void __launch_bounds__(kThreads) ssd_chunk_scan_kernel(const SsdParams p) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
-  const int N = p.N, H = p.H, L = p.L;
-  const int PN = pitch_n(N);
+  constexpr int PN = pitch_n(N);
+  constexpr int kMt = N / 16;                  // m16 tiles of the state rows
+  constexpr int kPg = kWarps / kMt;            // warps sharing one (1 or 2)
+  constexpr int kPj = 8 / kPg;                 // p tiles of a warp's state rows
+  const int H = p.H, L = p.L;
   const SsdLayout ly(N);
-  bf16* xs = reinterpret_cast<bf16*>(smem + ly.x);
-  bf16* xl = reinterpret_cast<bf16*>(smem + ly.xl);
-  bf16* bs = reinterpret_cast<bf16*>(smem + ly.b);
-  bf16* cs_t = reinterpret_cast<bf16*>(smem + ly.c);
   bf16* hs = reinterpret_cast<bf16*>(smem + ly.hs);
-  float* dts = reinterpret_cast<float*>(smem + ly.dt);
-  float* c2 = reinterpret_cast<float*>(smem + ly.cs);
+  bf16* ws = reinterpret_cast<bf16*>(smem + ly.w);
+  float* wrow = reinterpret_cast<float*>(smem + ly.wr);
   const int b = blockIdx.y, hd = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
-  const int C = H * kP + 2 * N;                  // conv channels
-  const long long ldx = 2LL * C;                  // split-pair row pitch
+  const int rb = warp & 3, hb = warp >> 2;     // output rows 16 rb.., p (and s) half hb
+  const int C = H * kP + 2 * N;                // conv channels
+  const long long ldx = 2LL * C;               // split-pair row pitch
   const float A2 = p.A[hd] * kLog2e, Dh = p.D[hd], bias = p.dt_bias[hd];
-  const int nrow = N / 4;                         // state rows per warp
-  const int ntm = nrow / 16;                      // their m16 tiles (1 or 2)
   float* hglob = p.h + (static_cast<long long>(b) * H + hd) * kP * N;   // [P][N]
 
-  // the state, fp32 in this warp's accumulators: tile (mi, pj) holds rows
-  // n = n0 + 16 mi + {g, g + 8}, columns p = 8 pj + 2 t4 + {0, 1}
-  float st[2][8][4];
-  const int n0 = warp * nrow;
+  // the state, fp32 in this warp's accumulators: tile pj holds rows
+  // n = 16 sm + {g, g + 8}, columns p = 8 (pj0 + pj) + 2 t4 + {0, 1}
+  const int sm = warp % kMt, pj0 = (warp / kMt) * kPj;
+  float st[kPj][4];
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
+  for (int pj = 0; pj < kPj; ++pj)
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int n = n0 + 16 * mi + g + (e >> 1) * 8, pp = 8 * pj + 2 * t4 + (e & 1);
-        st[mi][pj][e] = (mi < ntm && !p.zero_init) ? hglob[pp * N + n] : 0.0f;
-      }
+    for (int e = 0; e < 4; ++e) {
+      const int n = 16 * sm + g + (e >> 1) * 8, pp = 8 * (pj0 + pj) + 2 * t4 + (e & 1);
+      st[pj][e] = p.zero_init ? 0.0f : hglob[pp * N + n];
+    }
   auto store_state_copy = [&]() {
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi) {
-      if (mi >= ntm) break;
-#pragma unroll
-      for (int pj = 0; pj < 8; ++pj) {
-        const int n = n0 + 16 * mi + g, pp = 8 * pj + 2 * t4;
-        *reinterpret_cast<uint32_t*>(hs + n * kPitchP + pp) = pack2(st[mi][pj][0], st[mi][pj][1]);
-        *reinterpret_cast<uint32_t*>(hs + (n + 8) * kPitchP + pp) = pack2(st[mi][pj][2], st[mi][pj][3]);
-      }
+    for (int pj = 0; pj < kPj; ++pj) {
+      const int n = 16 * sm + g, pp = 8 * (pj0 + pj) + 2 * t4;
+      *reinterpret_cast<uint32_t*>(hs + n * kPitchP + pp) = pack2(st[pj][0], st[pj][1]);
+      *reinterpret_cast<uint32_t*>(hs + (n + 8) * kPitchP + pp) = pack2(st[pj][2], st[pj][3]);
     }
   };
   store_state_copy();
 
   const int nchunks = (L + kQ - 1) / kQ;
-  for (int ck = 0; ck < nchunks; ++ck) {
+  // warp 0 reads chunk ck's dt_raw (lane: tokens 2 lane, 2 lane + 1) one
+  // chunk before it turns them into dt and c
+  // (kept as raw bf16 until then: converting them here would wait for the loads)
+  bf16 draw[2] = {__float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f)};
+  auto fetch_dt = [&](int ck) {
+    if (warp != 0 || ck >= nchunks) return;
     const int t0 = ck * kQ, nt = min(kQ, L - t0);
-    // ---- the chunk's x (hi, lo), B, C (hi) rows; rows past L as zeros
-    {
-      const long long row0 = static_cast<long long>(b) * L + t0;
-      for (int i = tid; i < kQ * (kP / 8); i += kThreads) {          // x: 8 pieces of 8 per row
-        const int r = i / (kP / 8), k = i % (kP / 8);
-        if (r < nt) {
-          const bf16* src = p.xc + (row0 + r) * ldx + hd * kP + 8 * k;
-          cp16(xs + r * kPitchP + 8 * k, src);
-          cp16(xl + r * kPitchP + 8 * k, src + C);
-        } else {
-          *reinterpret_cast<uint4*>(xs + r * kPitchP + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(xl + r * kPitchP + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      const int np = N / 8;
-      for (int i = tid; i < kQ * np; i += kThreads) {                // B, C
-        const int r = i / np, k = i % np;
-        if (r < nt) {
-          const bf16* src = p.xc + (row0 + r) * ldx + H * kP + 8 * k;
-          cp16(bs + r * PN + 8 * k, src);
-          cp16(cs_t + r * PN + 8 * k, src + N);
-        } else {
-          *reinterpret_cast<uint4*>(bs + r * PN + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(cs_t + r * PN + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      if (warp == 0) {
-        // dt = softplus(dt_raw + bias), c_t log2(e) = A log2(e) cumsum(dt):
-        // lane holds tokens 2 lane, 2 lane + 1
-        float d[2];
+    const long long row0 = static_cast<long long>(b) * L + t0;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int r = 2 * lane + e;
-          d[e] = r < nt ? softplus(__bfloat162float(p.dt_raw[(row0 + r) * H + hd]) + bias) : 0.0f;
-        }
-        float s = d[0] + d[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float o = __shfl_up_sync(0xffffffffu, s, off);
-          if (lane >= off) s += o;
-        }
-        const float before = s - d[0] - d[1];
-        dts[2 * lane] = d[0];
-        dts[2 * lane + 1] = d[1];
-        c2[2 * lane] = A2 * (before + d[0]);
-        c2[2 * lane + 1] = A2 * s;
-      }
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      __syncthreads();
+    for (int e = 0; e < 2; ++e) {
+      const int r = 2 * lane + e;
+      if (r < nt) draw[e] = p.dt_raw[(row0 + r) * H + hd];
     }
+  };
+  // chunk ck's x (hi, lo), B, C (hi) rows into buffer `bi` (rows past L as
+  // zeros), and (from the fetched dt_raw) its dt = softplus(dt_raw + bias),
+  // c_t log2(e) = A log2(e) cumsum(dt)
+  auto load_chunk = [&](int ck, int bi) {
+    uint8_t* base = smem + bi * ly.buf;
+    bf16* xs_ = reinterpret_cast<bf16*>(base + ly.x);
+    bf16* xl_ = reinterpret_cast<bf16*>(base + ly.xl);
+    bf16* bs_ = reinterpret_cast<bf16*>(base + ly.b);
+    bf16* cs_ = reinterpret_cast<bf16*>(base + ly.c);
+    const int t0 = ck * kQ, nt = min(kQ, L - t0);
+    const long long row0 = static_cast<long long>(b) * L + t0;
+    for (int i = tid; i < kQ * (kP / 8); i += kThreads) {          // x: 8 pieces of 8 per row
+      const int r = i / (kP / 8), k = i % (kP / 8);
+      if (r < nt) {
+        const bf16* src = p.xc + (row0 + r) * ldx + hd * kP + 8 * k;
+        cp16(xs_ + r * kPitchP + 8 * k, src);
+        cp16(xl_ + r * kPitchP + 8 * k, src + C);
+      } else {
+        *reinterpret_cast<uint4*>(xs_ + r * kPitchP + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(xl_ + r * kPitchP + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    const int np = N / 8;
+    for (int i = tid; i < kQ * np; i += kThreads) {                // B, C
+      const int r = i / np, k = i % np;
+      if (r < nt) {
+        const bf16* src = p.xc + (row0 + r) * ldx + H * kP + 8 * k;
+        cp16(bs_ + r * PN + 8 * k, src);
+        cp16(cs_ + r * PN + 8 * k, src + N);
+      } else {
+        *reinterpret_cast<uint4*>(bs_ + r * PN + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(cs_ + r * PN + 8 * k) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (warp == 0) {
+      float* dts_ = reinterpret_cast<float*>(base + ly.dt);
+      float* c2_ = reinterpret_cast<float*>(base + ly.cs);
+      float d[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) d[e] = 2 * lane + e < nt ? softplus(__bfloat162float(draw[e]) + bias) : 0.0f;
+      float sum = d[0] + d[1];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, sum, off);
+        if (lane >= off) sum += o;
+      }
+      const float before = sum - d[0] - d[1];
+      dts_[2 * lane] = d[0];
+      dts_[2 * lane + 1] = d[1];
+      c2_[2 * lane] = A2 * (before + d[0]);
+      c2_[2 * lane + 1] = A2 * sum;
+    }
+  };
+  fetch_dt(0);
+  load_chunk(0, 0);
+  fetch_dt(1);
+  for (int ck = 0; ck < nchunks; ++ck) {
+    const int bi = ck & 1;
+    if (ck + 1 < nchunks) load_chunk(ck + 1, bi ^ 1);   // its buffer was freed by the barrier ending ck - 1
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    fetch_dt(ck + 2);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // chunk ck has landed
+    __syncthreads();
+    uint8_t* base = smem + bi * ly.buf;
+    const bf16* xs = reinterpret_cast<const bf16*>(base + ly.x);
+    const bf16* xl = reinterpret_cast<const bf16*>(base + ly.xl);
+    bf16* bs = reinterpret_cast<bf16*>(base + ly.b);
+    const bf16* cs_t = reinterpret_cast<const bf16*>(base + ly.c);
+    const float* dts = reinterpret_cast<const float*>(base + ly.dt);
+    const float* c2 = reinterpret_cast<const float*>(base + ly.cs);
+    const int t0 = ck * kQ, nt = min(kQ, L - t0);
     const float c2end = c2[kQ - 1];
+    const int r0 = 16 * rb;
 
-    // ---- output rows of this warp: Y = exp(c_t) C H_in + W X + D x
-    const int r0 = 16 * warp;
-    float y[8][4];
+    // ---- G = C B^T for rows r0.. and the s half hb, and the carry C H_in for
+    // rows r0.. and the p half hb, in one pass over K = N (shared A fragments)
+    float gacc[4][4], y[4][4];
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj) y[pj][0] = y[pj][1] = y[pj][2] = y[pj][3] = 0.0f;
-    for (int kk = 0; kk < N / 16; ++kk) {                          // carry: C (rows t) . H (K = N)
-      uint32_t a[4];
-      frag_a(a, cs_t, PN, r0, 16 * kk, lane);
-#pragma unroll
-      for (int pj = 0; pj < 8; pj += 2) {
-        uint32_t bb[4];
-        frag_b_t(bb, hs, kPitchP, 8 * pj, 16 * kk, lane);
-        mma(y[pj], a, bb[0], bb[1]);
-        mma(y[pj + 1], a, bb[2], bb[3]);
-      }
+    for (int j = 0; j < 4; ++j) {
+      gacc[j][0] = gacc[j][1] = gacc[j][2] = gacc[j][3] = 0.0f;
+      y[j][0] = y[j][1] = y[j][2] = y[j][3] = 0.0f;
     }
-    const float eg = ex2_approx(c2[r0 + g]), eg8 = ex2_approx(c2[r0 + g + 8]);
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj) {
-      y[pj][0] *= eg; y[pj][1] *= eg; y[pj][2] *= eg8; y[pj][3] *= eg8;
-    }
-    // G = C B^T for rows t, all s; then W = G exp(c_t - c_s) dt_s (s <= t)
-    float gacc[8][4];
-#pragma unroll
-    for (int sj = 0; sj < 8; ++sj) gacc[sj][0] = gacc[sj][1] = gacc[sj][2] = gacc[sj][3] = 0.0f;
     for (int kk = 0; kk < N / 16; ++kk) {
-      uint32_t a[4];
+      uint32_t a[4], bb[2][4], hh[2][4];
       frag_a(a, cs_t, PN, r0, 16 * kk, lane);
+      frag_b(bb[0], bs, PN, 32 * hb, 16 * kk, lane);
+      frag_b(bb[1], bs, PN, 32 * hb + 16, 16 * kk, lane);
+      frag_b_t(hh[0], hs, kPitchP, 32 * hb, 16 * kk, lane);
+      frag_b_t(hh[1], hs, kPitchP, 32 * hb + 16, 16 * kk, lane);
 #pragma unroll
-      for (int sj = 0; sj < 8; sj += 2) {
-        uint32_t bb[4];
-        frag_b(bb, bs, PN, 8 * sj, 16 * kk, lane);
-        mma(gacc[sj], a, bb[0], bb[1]);
-        mma(gacc[sj + 1], a, bb[2], bb[3]);
+      for (int q = 0; q < 2; ++q) {
+        mma(gacc[2 * q], a, bb[q][0], bb[q][1]);
+        mma(gacc[2 * q + 1], a, bb[q][2], bb[q][3]);
+        mma(y[2 * q], a, hh[q][0], hh[q][1]);
+        mma(y[2 * q + 1], a, hh[q][2], hh[q][3]);
       }
     }
-    uint32_t wa[4][4];
+    // W = G exp(c_t - c_s) dt_s (s <= t) into shared memory; carry rows scaled
+    // by exp(c_t)
     {
       const int ta = r0 + g, tb = ta + 8;
       const float cta = c2[ta], ctb = c2[tb];
 #pragma unroll
-      for (int sj = 0; sj < 8; ++sj) {
-        const int s0 = 8 * sj + 2 * t4, s1 = s0 + 1;
+      for (int sj = 0; sj < 4; ++sj) {
+        const int s0 = 32 * hb + 8 * sj + 2 * t4, s1 = s0 + 1;
         const float w0a = s0 <= ta ? ex2_approx(cta - c2[s0]) * dts[s0] : 0.0f;
         const float w1a = s1 <= ta ? ex2_approx(cta - c2[s1]) * dts[s1] : 0.0f;
         const float w0b = s0 <= tb ? ex2_approx(ctb - c2[s0]) * dts[s0] : 0.0f;
         const float w1b = s1 <= tb ? ex2_approx(ctb - c2[s1]) * dts[s1] : 0.0f;
-        const uint32_t top = pack2(gacc[sj][0] * w0a, gacc[sj][1] * w1a);
-        const uint32_t bot = pack2(gacc[sj][2] * w0b, gacc[sj][3] * w1b);
-        // A fragment of k-step sj / 2: regs 0, 1 from n-tile 2kk, regs 2, 3 from 2kk + 1
-        wa[sj >> 1][(sj & 1) * 2 + 0] = top;
-        wa[sj >> 1][(sj & 1) * 2 + 1] = bot;
+        *reinterpret_cast<uint32_t*>(ws + ta * kPitchP + s0) = pack2(gacc[sj][0] * w0a, gacc[sj][1] * w1a);
+        *reinterpret_cast<uint32_t*>(ws + tb * kPitchP + s0) = pack2(gacc[sj][2] * w0b, gacc[sj][3] * w1b);
+      }
+      const float eg = ex2_approx(cta), eg8 = ex2_approx(ctb);
+#pragma unroll
+      for (int pj = 0; pj < 4; ++pj) {
+        y[pj][0] *= eg; y[pj][1] *= eg; y[pj][2] *= eg8; y[pj][3] *= eg8;
       }
     }
+    // the state weights exp(c_end - c_s) dt_s of this chunk
+    if (tid < kQ) wrow[tid] = ex2_approx(c2end - c2[tid]) * dts[tid];
+    __syncthreads();   // W complete
+    // ---- intra-chunk: y += W X (K = s)
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {                                // Y += W X (K = s)
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a[4], bb[2][4];
+      frag_a(a, ws, kPitchP, r0, 16 * kk, lane);
+      frag_b_t(bb[0], xs, kPitchP, 32 * hb, 16 * kk, lane);
+      frag_b_t(bb[1], xs, kPitchP, 32 * hb + 16, 16 * kk, lane);
 #pragma unroll
-      for (int pj = 0; pj < 8; pj += 2) {
-        uint32_t bb[4];
-        frag_b_t(bb, xs, kPitchP, 8 * pj, 16 * kk, lane);
-        mma(y[pj], wa[kk], bb[0], bb[1]);
-        mma(y[pj + 1], wa[kk], bb[2], bb[3]);
+      for (int q = 0; q < 2; ++q) {
+        mma(y[2 * q], a, bb[q][0], bb[q][1]);
+        mma(y[2 * q + 1], a, bb[q][2], bb[q][3]);
       }
     }
     {
       const int ta = r0 + g, tb = ta + 8;
       const long long rowa = static_cast<long long>(b) * L + t0 + ta, rowb = rowa + 8;
 #pragma unroll
-      for (int pj = 0; pj < 8; ++pj) {
-        const int pp = 8 * pj + 2 * t4;
+      for (int pj = 0; pj < 4; ++pj) {
+        const int pp = 32 * hb + 8 * pj + 2 * t4;
         if (ta < nt) {
           const float2 xh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xs + ta * kPitchP + pp));
           const float2 xo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(xl + ta * kPitchP + pp));
@@ -312,57 +344,52 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_scan_kernel(const SsdParam
         }
       }
     }
-    __syncthreads();   // every warp is done with B (raw) and the state copy
-
-    // ---- B scaled by exp(c_end - c_s) dt_s, in place
-    for (int i = tid; i < kQ * (N / 2); i += kThreads) {
-      const int r = i / (N / 2), k = 2 * (i % (N / 2));
-      const float w = ex2_approx(c2end - c2[r]) * dts[r];
-      __nv_bfloat162* q = reinterpret_cast<__nv_bfloat162*>(bs + r * PN + k);
-      const float2 v = __bfloat1622float2(*q);
-      *q = __floats2bfloat162_rn(v.x * w, v.y * w);
-    }
-    __syncthreads();
-    // ---- state: H = exp(c_end) H + (B scaled)^T X for this warp's rows n
-    const float eend = ex2_approx(c2end);
+    // ---- state: H = exp(c_end) H + (B scaled)^T X for this warp's tiles, B
+    // scaled by exp(c_end - c_s) dt_s in the A fragments (k = s)
+    {
+      const float eend = ex2_approx(c2end);
+      float sacc[kPj][4];
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi) {
-      if (mi >= ntm) break;
-      float sacc[8][4];
-#pragma unroll
-      for (int pj = 0; pj < 8; ++pj) sacc[pj][0] = sacc[pj][1] = sacc[pj][2] = sacc[pj][3] = 0.0f;
+      for (int pj = 0; pj < kPj; ++pj) sacc[pj][0] = sacc[pj][1] = sacc[pj][2] = sacc[pj][3] = 0.0f;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         uint32_t a[4];
-        frag_a_t(a, bs, PN, n0 + 16 * mi, 16 * kk, lane);
+        frag_a_t(a, bs, PN, 16 * sm, 16 * kk, lane);
+        {
+          // a[0], a[1]: k = 16 kk + 2 t4 + {0, 1}; a[2], a[3]: k + 8
+          const float2 wlo = *reinterpret_cast<const float2*>(wrow + 16 * kk + 2 * t4);
+          const float2 whi = *reinterpret_cast<const float2*>(wrow + 16 * kk + 8 + 2 * t4);
 #pragma unroll
-        for (int pj = 0; pj < 8; pj += 2) {
+          for (int r = 0; r < 4; ++r) {
+            const float2 wv = r < 2 ? wlo : whi;
+            const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a[r]));
+            a[r] = pack2(v.x * wv.x, v.y * wv.y);
+          }
+        }
+#pragma unroll
+        for (int pj = 0; pj < kPj; pj += 2) {
           uint32_t bb[4];
-          frag_b_t(bb, xs, kPitchP, 8 * pj, 16 * kk, lane);
+          frag_b_t(bb, xs, kPitchP, 8 * (pj0 + pj), 16 * kk, lane);
           mma(sacc[pj], a, bb[0], bb[1]);
           mma(sacc[pj + 1], a, bb[2], bb[3]);
         }
       }
 #pragma unroll
-      for (int pj = 0; pj < 8; ++pj)
+      for (int pj = 0; pj < kPj; ++pj)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st[mi][pj][e] = fmaf(eend, st[mi][pj][e], sacc[pj][e]);
+        for (int e = 0; e < 4; ++e) st[pj][e] = fmaf(eend, st[pj][e], sacc[pj][e]);
     }
     store_state_copy();
-    __syncthreads();   // state copy complete; x, B, C free for the next chunk
+    __syncthreads();   // state copy complete; this buffer free for chunk ck + 2
   }
   // final state
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi) {
-    if (mi >= ntm) break;
+  for (int pj = 0; pj < kPj; ++pj)
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int n = n0 + 16 * mi + g + (e >> 1) * 8, pp = 8 * pj + 2 * t4 + (e & 1);
-        hglob[pp * N + n] = st[mi][pj][e];
-      }
-  }
+    for (int e = 0; e < 4; ++e) {
+      const int n = 16 * sm + g + (e >> 1) * 8, pp = 8 * (pj0 + pj) + 2 * t4 + (e & 1);
+      hglob[pp * N + n] = st[pj][e];
+    }
 }
 
 // The conv state after a prompt: the last K raw inputs of every channel
