@@ -49,7 +49,7 @@ from gated_memory_sharing_b200 import synth  # noqa: E402
 
 HEADLINE = "prefill_b1_l2048"
 WORKLOADS = ("prefill_b1_l2048", "decode_b64", "long_prefill_b4_l32768", "sharing_b2_l8192",
-             "sharing_decode_b16", "cross_attn_vs_gmu_b64")
+             "sharing_decode_b16", "cross_attn_vs_gmu_b64", "sambay2_prefill_b1_l2048")
 UNIT = "tokens/s"
 METRICS = {
     "prefill_b1_l2048": "scan+GMU prefill tokens/s",
@@ -58,6 +58,7 @@ METRICS = {
     "sharing_b2_l8192": "scan+8xGMU prefill tokens/s",
     "sharing_decode_b16": "scan+8xGMU decode tokens/s",
     "cross_attn_vs_gmu_b64": "cross-attention decode tokens/s at 2048 cached tokens",
+    "sambay2_prefill_b1_l2048": "SambaY-2 (Mamba-2 SSD) memory readout prefill tokens/s",
 }
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from an
 # earlier ncu capture of the headline workload, for kernels unchanged since
@@ -214,6 +215,8 @@ def dev_normal(shape, seed, device):
 
 def workload_dims(name):
     """(dims, seed, gmu layers, decode?) of a bench workload."""
+    if name == "sambay2_prefill_b1_l2048":
+        return synth.SSD_WORKLOAD, synth.SSD_WORKLOAD_SEED, 0, False
     if name == "cross_attn_vs_gmu_b64":
         d, seed = synth.workload("decode_b64")
         return d, seed, 1, False
@@ -229,6 +232,9 @@ def workload_dims(name):
 
 
 def config_of(name, d, layers, decode):
+    if name == "sambay2_prefill_b1_l2048":
+        return {"workload": name, "batch": d.batch, "seq_len": d.seqlen, "nheads": d.nheads, "headdim": d.headdim,
+                "d_inner": d.nheads * d.headdim, "d_state": d.d_state, "d_conv": d.d_conv, "ngroups": 1}
     c = {"workload": name, "batch": d.batch, "seq_len": d.seqlen, "d_model": d.d_model,
          "d_inner": d.d_inner, "d_state": d.d_state, "d_conv": d.d_conv, "dt_rank": d.dt_rank,
          "gmu_layers": layers}
@@ -258,6 +264,19 @@ def cpu_baseline(name, budget_s=8.0, reps_max=4):
     from oracle import sambay_ref as ref
     d, seed, layers, decode = workload_dims(name)
     cores = len(os.sched_getaffinity(0))
+    if name == "sambay2_prefill_b1_l2048":
+        from oracle import ssd_ref
+        L = 128
+        w = synth.ssd_weights(d, seed)
+        xbc, dt_raw = synth.ssd_inputs(d, seed, seqlen=L)
+        reps, t0 = 0, time.perf_counter()
+        while reps < reps_max and (reps == 0 or time.perf_counter() - t0 < budget_s):
+            ssd_ref.mamba2_scan_ref(xbc, dt_raw, w)
+            reps += 1
+        el = time.perf_counter() - t0
+        return {"value": reps * L / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"the first {L} tokens of the sequence (conv + SSD recurrence, all {d.nheads} heads) "
+                          f"x {reps}, {el:.1f} s of float64 NumPy"}
     if name == "cross_attn_vs_gmu_b64":
         S, N = 4, d.seqlen
         q, K, V = synth.attention_inputs(S, N, synth.ATTN_Q_HEADS, synth.ATTN_KV_HEADS, synth.ATTN_HEAD_DIM, seed)
@@ -651,6 +670,89 @@ def bench_decode(args, ctx, name):
     }
 
 
+# --------------------------------------------------------------------- our arm: SambaY-2 prefill
+
+def bench_ssd(args, ctx, name):
+    """The SambaY-2 variant's memory readout over a prompt: conv over
+    [x | B | C], softplus dt, and the chunked Mamba-2 SSD scan."""
+    import torch
+    from gated_memory_sharing_b200 import abi
+    from gated_memory_sharing_b200.layers import Mamba2Scan
+    world, rank, device, flush, stream, peaks, peak_kind, sms = ctx
+    d, seed, _, _ = workload_dims(name)
+    layer = Mamba2Scan(synth.ssd_weights(d, seed))
+    rs = seed + 7919 * rank
+    xbc = dev_normal((d.batch, d.seqlen, d.channels), rs, device)
+    dt_raw = (0.5 * dev_normal((d.batch, d.seqlen, d.nheads), rs + 1, device).float()).to(torch.bfloat16)
+    M, h, cs = layer.prefill(xbc, dt_raw)
+
+    def step():
+        layer.prefill(xbc, dt_raw, h, cs, M=M, fresh=True)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush(i)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    ms = total_ms / steps
+    per_kernel = {}
+    for i in range(3):
+        flush(i)
+        with abi.KernelTimer(max_launches=16) as kt:
+            step()
+        torch.cuda.synchronize()
+        launches = len(kt.names)
+        for kname, kms in kt.durations_ms():
+            per_kernel.setdefault(kname, []).append(1e3 * kms)
+    kernels_us = {k: statistics.mean(v) for k, v in per_kernel.items()}
+    # algorithmic bytes: the in_proj slices in, M out, the fp32 state in and
+    # out, the conv window; the weights are a few KB
+    T, P, N, H = d.batch * d.seqlen, d.headdim, d.d_state, d.nheads
+    nbytes = T * d.channels * 2 + T * H * 2 + T * H * P * 2 + 2 * d.batch * H * P * N * 4
+    achieved = nbytes / (ms / 1e3) / 1e9
+    # end to end: the in_proj slices from pinned host memory in, M back out
+    xh = xbc.cpu().pin_memory()
+    dh = dt_raw.cpu().pin_memory()
+    mh = torch.empty(M.shape, dtype=M.dtype).pin_memory()
+    xd, dd = torch.empty_like(xbc), torch.empty_like(dt_raw)
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    torch.cuda.synchronize()
+    e2e_ev[0].record(stream)
+    for _ in range(steps):
+        xd.copy_(xh, non_blocking=True)
+        dd.copy_(dh, non_blocking=True)
+        layer.prefill(xd, dd, h, cs, M=M, fresh=True)
+        mh.copy_(M, non_blocking=True)
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]), world, device)
+    dom = max(kernels_us.items(), key=lambda kv: kv[1])
+    return {
+        "metric": METRICS[name], "value": world * T / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+        "steps": steps, "config": config_of(name, d, 0, False),
+        "l2": "flushed before every timed step (256 MB write + 256 MB read, outside the step events)",
+        "kernels_us": kernels_us,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "algorithmic_bytes_per_step": nbytes,
+                     "kernel": "whole SambaY-2 readout (conv + SSD scan + conv state)",
+                     "dominant_kernel": dom[0], "dominant_kernel_us": dom[1], "peak_note": f"{peak_kind} HBM copy"},
+        "e2e": {"value": world * steps * T / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": (xbc.numel() + dt_raw.numel()) * 2, "d2h_bytes_per_step": M.numel() * 2},
+        "gpu_launches": launches * steps,
+    }
+
+
 # --------------------------------------------------------------------- our arm: attention vs GMU
 
 def bench_attn_vs_gmu(args, ctx, name):
@@ -753,6 +855,9 @@ def run_ours(args, world, rank, local):
     for name in names:
         if name == "cross_attn_vs_gmu_b64":
             results[name] = bench_attn_vs_gmu(args, ctx, name)
+            continue
+        if name == "sambay2_prefill_b1_l2048":
+            results[name] = bench_ssd(args, ctx, name)
             continue
         fn = bench_decode if workload_dims(name)[3] else bench_prefill
         results[name] = fn(args, ctx, name)
