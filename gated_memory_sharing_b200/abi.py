@@ -48,6 +48,8 @@ EXPORTS = (
     "sambay_cross_attn_decode",
     "sambay_ssd_prefill_workspace",
     "sambay_ssd_prefill",
+    "sambay_ssd_step_workspace",
+    "sambay_ssd_step",
     "sambay_gmu_step_stall_test",
     "sambay_profile_begin",
     "sambay_profile_end",
@@ -165,6 +167,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sambay_cross_attn_decode": (ctypes.c_int, [pa, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp]),
         "sambay_ssd_prefill_workspace": (sz, [psd]),
         "sambay_ssd_prefill": (ctypes.c_int, [psw, psd, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "sambay_ssd_step_workspace": (sz, [psd]),
+        "sambay_ssd_step": (ctypes.c_int, [psw, psd, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sambay_decode_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, i32, pg, vp, vp, sz, vp]),
         "sambay_gmu_step_stall_test": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz,
                                                       ctypes.c_uint64, vp]),
@@ -283,6 +287,17 @@ def sambay_ssd_prefill(w: SsdWeights, dims: SsdDims, xbc, dt_raw, M, ssm_state, 
     _check("sambay_ssd_prefill", load().sambay_ssd_prefill(
         ctypes.byref(w), ctypes.byref(dims), _p(xbc), _p(dt_raw), _p(M), _p(ssm_state), _p(conv_state),
         1 if zero_init else 0, _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_ssd_step_workspace(dims: SsdDims) -> int:
+    return load().sambay_ssd_step_workspace(ctypes.byref(dims))
+
+
+def sambay_ssd_step(w: SsdWeights, dims: SsdDims, xbc_t, dt_raw_t, m_t, ssm_state, conv_state, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_ssd_step", load().sambay_ssd_step(
+        ctypes.byref(w), ctypes.byref(dims), _p(xbc_t), _p(dt_raw_t), _p(m_t), _p(ssm_state), _p(conv_state),
+        _p(ws), ws_bytes, _stream(stream)))
 
 
 def sambay_decode_step_workspace(dims: Dims, n_layers: int) -> int:

@@ -1519,6 +1519,43 @@ sambay_status sambay_ssd_prefill(const sambay_ssd_weights* w, const sambay_ssd_d
   return SAMBAY_OK;
 }
 
+size_t sambay_ssd_step_workspace(const sambay_ssd_dims* d) {
+  if (ssd_check(d) != SAMBAY_OK) return 0;
+  const size_t C = static_cast<size_t>(d->nheads) * d->headdim + 2 * static_cast<size_t>(d->d_state);
+  return round256(static_cast<size_t>(d->batch) * C * 4);
+}
+
+sambay_status sambay_ssd_step(const sambay_ssd_weights* w, const sambay_ssd_dims* d, const void* xbc_t,
+                              const void* dt_raw_t, void* m_t, float* ssm_state, void* conv_state, void* ws,
+                              size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(ssd_check(d));
+  if (!w) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({w->conv_w, w->conv_b, w->dt_bias, w->A, w->D}));
+  SAMBAY_TRY(check_ptrs({xbc_t, dt_raw_t, m_t, ssm_state, conv_state}));
+  if (m_t == xbc_t) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_ssd_step_workspace(d)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int C = d->nheads * d->headdim + 2 * d->d_state;
+  float* xc = static_cast<float*>(ws);
+  {
+    const long long n = static_cast<long long>(d->batch) * (C / 8);
+    ProfScope ps("ssd_step_conv", st);
+    sambay::ssd::ssd_step_conv_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        static_cast<const bf16*>(xbc_t), static_cast<bf16*>(conv_state), static_cast<const bf16*>(w->conv_w),
+        static_cast<const bf16*>(w->conv_b), xc, d->batch, C);
+    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+  }
+  auto kern = d->d_state == 128 ? sambay::ssd::ssd_step_kernel<128> : sambay::ssd::ssd_step_kernel<64>;
+  ProfScope ps("ssd_step", st);
+  return launch_k(kern, dim3(d->nheads, d->batch), dim3(256), 0, st, true, 1, static_cast<const float*>(xc),
+                  static_cast<const bf16*>(dt_raw_t), w->dt_bias, w->A, w->D, ssm_state, static_cast<bf16*>(m_t),
+                  d->nheads) == cudaSuccess
+             ? SAMBAY_OK
+             : SAMBAY_ERR_CUDA;
+}
+
 sambay_status sambay_scan_step_noalloc(const sambay_scan_weights* w, const sambay_dims* d,
                                        const void* u_t, void* m_t, float* ssm_state,
                                        void* conv_state, sambay_stream_t stream) {

@@ -416,5 +416,102 @@ __global__ void conv_state_update_kernel(const bf16* __restrict__ u, bf16* __res
   for (int k = 0; k < K; ++k) cs[k] = nw[k];
 }
 
+// ------------------------------------------------------------------ decode step
+//
+// One token per sequence, the state updated in place (constant size: the
+// decode state of [Notes] 方法详解 > 关键设计 for this variant).  Two kernels:
+// the conv step over [x | B | C] (window shifted in place, output fp32 in the
+// workspace), then the SSD update per (head, sequence).
+
+// Thread: 8 channels of one sequence.
+__global__ void __launch_bounds__(256) ssd_step_conv_kernel(const bf16* __restrict__ xbc_t,
+                                                            bf16* __restrict__ conv_state,
+                                                            const bf16* __restrict__ conv_w,
+                                                            const bf16* __restrict__ conv_b,
+                                                            float* __restrict__ xc, int Bt, int C) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int K = 4;
+  const long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  const int groups = C / 8;
+  if (i >= static_cast<long long>(Bt) * groups) return;
+  const int b = static_cast<int>(i / groups), c0 = static_cast<int>(i % groups) * 8;
+  const long long off = static_cast<long long>(b) * C + c0;
+  Pack16 in, bias, win[4], wt[4];
+  in.u = *reinterpret_cast<const uint4*>(xbc_t + off);
+  bias.u = *reinterpret_cast<const uint4*>(conv_b + c0);
+  uint4* wp = reinterpret_cast<uint4*>(conv_state + off * K);
+  const uint4* kp = reinterpret_cast<const uint4*>(conv_w + static_cast<long long>(c0) * K);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    win[j].u = wp[j];
+    wt[j].u = kp[j];
+  }
+  bf16* wv = reinterpret_cast<bf16*>(win);      // [8 channels][K], oldest first
+  const bf16* kv = reinterpret_cast<const bf16*>(wt);
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int k = 0; k < K - 1; ++k) wv[e * K + k] = wv[e * K + k + 1];
+    wv[e * K + K - 1] = in.h[e];
+    float acc = __bfloat162float(bias.h[e]);
+#pragma unroll
+    for (int k = 0; k < K; ++k) acc = fmaf(__bfloat162float(kv[e * K + k]), __bfloat162float(wv[e * K + k]), acc);
+    y[e] = silu(acc);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) wp[j] = win[j].u;
+  float4* o = reinterpret_cast<float4*>(xc + off);
+  o[0] = make_float4(y[0], y[1], y[2], y[3]);
+  o[1] = make_float4(y[4], y[5], y[6], y[7]);
+}
+
+// CTA (head, sequence), 256 threads: thread (p = tid / 4, q = tid % 4) owns
+// the states n = 4 (q + 4 j) + {0..3} of channel p (the 4 threads of a
+// channel read 64 contiguous bytes per step), as 16-byte pieces; the readout
+// sums the 4 threads' parts with two shuffles.
+template <int N>
+__global__ void __launch_bounds__(256) ssd_step_kernel(const float* __restrict__ xc, const bf16* __restrict__ dt_raw,
+                                                       const float* __restrict__ dt_bias, const float* __restrict__ A,
+                                                       const float* __restrict__ D, float* __restrict__ h,
+                                                       bf16* __restrict__ m_t, int H) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int NQ = N / 4;
+  __shared__ __align__(16) float bc_s[2 * N];
+  const int hd = blockIdx.x, b = blockIdx.y;
+  const int C = H * kP + 2 * N;
+  const float* row = xc + static_cast<long long>(b) * C;
+  for (int i = threadIdx.x; i < 2 * N; i += blockDim.x) bc_s[i] = row[H * kP + i];
+  const float dt = softplus(__bfloat162float(dt_raw[static_cast<long long>(b) * H + hd]) + dt_bias[hd]);
+  const float a = ex2_approx(dt * A[hd] * kLog2e);
+  const int pch = threadIdx.x >> 2, q = threadIdx.x & 3;
+  const float x = row[hd * kP + pch];
+  const float dx = dt * x;
+  __syncthreads();
+  float* hp = h + ((static_cast<long long>(b) * H + hd) * kP + pch) * N;
+  float y = 0.0f;
+#pragma unroll
+  for (int jj = 0; jj < NQ / 4; ++jj) {
+    const int n0 = 4 * (q + 4 * jj);
+    float4 v = *reinterpret_cast<const float4*>(hp + n0);
+    const float4 bb = *reinterpret_cast<const float4*>(bc_s + n0);
+    const float4 cc = *reinterpret_cast<const float4*>(bc_s + N + n0);
+    v.x = fmaf(a, v.x, dx * bb.x);
+    v.y = fmaf(a, v.y, dx * bb.y);
+    v.z = fmaf(a, v.z, dx * bb.z);
+    v.w = fmaf(a, v.w, dx * bb.w);
+    y = fmaf(cc.x, v.x, y);
+    y = fmaf(cc.y, v.y, y);
+    y = fmaf(cc.z, v.z, y);
+    y = fmaf(cc.w, v.w, y);
+    *reinterpret_cast<float4*>(hp + n0) = v;
+  }
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  y += __shfl_xor_sync(0xffffffffu, y, 2);
+  if (q == 0) m_t[static_cast<long long>(b) * H * kP + hd * kP + pch] = __float2bfloat16_rn(fmaf(D[hd], x, y));
+}
+
 }  // namespace ssd
 }  // namespace sambay

@@ -275,3 +275,17 @@ class Mamba2Scan:
             self._ws[(B, L)] = ws
         abi.sambay_ssd_prefill(self.abi_w, d, xbc, dt_raw, M, ssm_state, conv_state, fresh, ws, stream)
         return M, ssm_state, conv_state
+
+    def step(self, xbc_t, dt_raw_t, ssm_state, conv_state, m_t=None, stream=None):
+        """xbc_t [B, C], dt_raw_t [B, H] -> m_t [B, H * P]; states updated in place."""
+        B = xbc_t.shape[0]
+        if m_t is None:
+            m_t = torch.empty(B, self.nheads * self.headdim, dtype=self.dtype, device=self.device)
+        d = self.dims(B, 1)
+        n = abi.sambay_ssd_step_workspace(d)
+        ws = self._ws.get(("step", B))
+        if ws is None:
+            ws = workspace(n, self.device)
+            self._ws[("step", B)] = ws
+        abi.sambay_ssd_step(self.abi_w, d, xbc_t, dt_raw_t, m_t, ssm_state, conv_state, ws, stream)
+        return m_t

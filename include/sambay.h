@@ -374,6 +374,23 @@ SAMBAY_API sambay_status sambay_ssd_prefill(const sambay_ssd_weights* w, const s
                                             sambay_stream_t stream);
 
 /*
+ * sambay_ssd_step - one decode token per sequence of the SambaY-2 memory:
+ * the prompt readout with L = 1 on the carried states, both updated IN
+ * PLACE (the conv window shifted, the SSD state advanced).  Two kernels: the
+ * conv step over [x | B | C] (fp32 output in ws), then the state update per
+ * (head, sequence).  dims->seqlen is ignored.
+ *
+ *   xbc_t [Bt, C] io in;  dt_raw_t [Bt, H] io in;  m_t [Bt, H*P] io out
+ *   (must not alias xbc_t);  ssm_state [Bt, H, P, N] f32 in/out;
+ *   conv_state [Bt, C, K] io in/out.  Sizes as for sambay_ssd_prefill.
+ *   ws: >= sambay_ssd_step_workspace(dims) = Bt * C * 4 bytes (rounded).
+ */
+SAMBAY_API size_t sambay_ssd_step_workspace(const sambay_ssd_dims* dims);
+SAMBAY_API sambay_status sambay_ssd_step(const sambay_ssd_weights* w, const sambay_ssd_dims* dims,
+                                         const void* xbc_t, const void* dt_raw_t, void* m_t, float* ssm_state,
+                                         void* conv_state, void* ws, size_t ws_bytes, sambay_stream_t stream);
+
+/*
  * sambay_scan_step_noalloc - sambay_scan_step for callers that cannot
  * allocate device memory.  The paper has no counterpart; this is a property
  * of the library, not of the method.

@@ -32,7 +32,7 @@ def _run(d, seed, seqlen=None):
     (2, 77, 2, 64),       # two partial chunks, ragged tail
     (1, 64, 3, 128),      # exactly one chunk
     (3, 200, 2, 128),     # several chunks, a 8-token tail
-    (1, 5, 4, 64),        # shorter than a chunk and than... the conv window + 1
+    (1, 5, 4, 64),        # shorter than a chunk, one token past the conv window
 ])
 def test_ssd_prefill_matches_oracle(B, L, H, N):
     d = synth.SsdDims(B, L, H, 64, N)
@@ -105,3 +105,52 @@ def test_ssd_prefill_repeatable():
     M2, h2, _ = layer.prefill(to_device(xbc, abi.BF16), to_device(dt_raw, abi.BF16))
     torch.cuda.synchronize()
     assert torch.equal(M, M2) and torch.equal(h, h2)
+
+
+@pytest.mark.parametrize("B,H,N", [(3, 2, 128), (2, 3, 64)])
+def test_ssd_decode_steps_equal_oracle_prefill(B, H, N):
+    """Decode steps after a prompt (states updated in place) against the
+    oracle's readout of the whole token sequence."""
+    d = synth.SsdDims(B, 40, H, 64, N)
+    seed = 60 + B + N
+    w = synth.ssd_weights(d, seed)
+    xbc, dt_raw = synth.ssd_inputs(d, seed)
+    layer = Mamba2Scan(w)
+    L0 = 33
+    _, h, cs = layer.prefill(to_device(xbc[:, :L0], abi.BF16), to_device(dt_raw[:, :L0], abi.BF16))
+    r = ssd_ref.mamba2_scan_ref(xbc, dt_raw, w)
+    for t in range(L0, d.seqlen):
+        m = layer.step(to_device(np.ascontiguousarray(xbc[:, t]), abi.BF16),
+                       to_device(np.ascontiguousarray(dt_raw[:, t]), abi.BF16), h, cs)
+        torch.cuda.synchronize()
+        assert_close(host(m), r["M"][:, t], TOL_BF16, f"step {t}")
+    assert_close(host(h), r["ssm_state"], TOL_BF16, "state after steps")
+    np.testing.assert_array_equal(host(cs), r["conv_state"])
+
+
+def test_ssd_decode_b64_full_width_sampled_heads():
+    """64 sequences at 80 heads of 64, d_state 128: a short prompt, then decode
+    steps; three heads of every sequence against the oracle."""
+    d = synth.SsdDims(64, 20, 80, 64, 128)
+    seed = 70
+    w = synth.ssd_weights(d, seed)
+    xbc, dt_raw = synth.ssd_inputs(d, seed)
+    layer = Mamba2Scan(w)
+    L0 = 16
+    _, h, cs = layer.prefill(to_device(xbc[:, :L0], abi.BF16), to_device(dt_raw[:, :L0], abi.BF16))
+    ms = []
+    for t in range(L0, d.seqlen):
+        ms.append(host(layer.step(to_device(np.ascontiguousarray(xbc[:, t]), abi.BF16),
+                                  to_device(np.ascontiguousarray(dt_raw[:, t]), abi.BF16), h, cs)))
+    torch.cuda.synchronize()
+    P, N, H = d.headdim, d.d_state, d.nheads
+    heads = [1, 40, H - 1]
+    cols = np.concatenate([np.arange(k * P, (k + 1) * P) for k in heads] + [np.arange(H * P, H * P + 2 * N)])
+    ws = dict(w)
+    ws["conv_w"], ws["conv_b"] = w["conv_w"][cols], w["conv_b"][cols]
+    for k in ("dt_bias", "A", "D"):
+        ws[k] = w[k][heads]
+    r = ssd_ref.mamba2_scan_ref(xbc[..., cols], dt_raw[..., heads], ws)
+    got = np.stack(ms, axis=1).reshape(64, d.seqlen - L0, H, P)[:, :, heads].reshape(64, d.seqlen - L0, -1)
+    assert_close(got, r["M"][:, L0:], TOL_BF16, "decode m_t (sampled heads)")
+    assert_close(host(h)[:, heads], r["ssm_state"], TOL_BF16, "state (sampled heads)")
