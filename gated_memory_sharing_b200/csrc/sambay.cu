@@ -1149,11 +1149,11 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
   float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
-  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 8, true>(
+  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 4, true>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, false,
       true, tail, L.tail_bytes, "gmu_gate_tail")));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
-  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 8, true>(
+  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 4, true>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st, true, true, tail, L.tail_bytes, "gmu_out_tail")));
   return SAMBAY_OK;
