@@ -34,9 +34,13 @@ EXPORTS = (
     "gmu_forward_workspace",
     "gmu_step_workspace",
     "sambay_scan_prefill",
+    "sambay_scan_prefill_xproj",
+    "sambay_scan_prefill_finish",
     "sambay_scan_step",
     "sambay_scan_step_noalloc",
     "gmu_forward",
+    "gmu_forward_partial",
+    "gmu_finish",
     "gmu_step",
     "sambay_in_proj_workspace",
     "sambay_in_proj",
@@ -154,9 +158,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gmu_forward_workspace": (sz, [pd, i64]),
         "gmu_step_workspace": (sz, [pd, i64]),
         "sambay_scan_prefill": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]),
+        "sambay_scan_prefill_xproj": (ctypes.c_int, [pw, pd, vp, vp, ctypes.c_int, vp, vp, sz, vp]),
+        "sambay_scan_prefill_finish": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]),
         "sambay_scan_step": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp, sz, vp]),
         "sambay_scan_step_noalloc": (ctypes.c_int, [pw, pd, vp, vp, vp, vp, vp]),
         "gmu_forward": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "gmu_forward_partial": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "gmu_finish": (ctypes.c_int, [pd, i64, vp, vp, vp, vp]),
         "gmu_step": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sambay_in_proj_workspace": (sz, [pd, i64]),
         "sambay_in_proj": (ctypes.c_int, [pd, i64, vp, vp, vp, vp, sz, vp]),
@@ -236,6 +244,22 @@ def sambay_scan_prefill(weights: ScanWeights, dims: Dims, u, M, ssm_state, conv_
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("sambay_scan_prefill", load().sambay_scan_prefill(
         ctypes.byref(weights), ctypes.byref(dims), _p(u), _p(M), _p(ssm_state), _p(conv_state),
+        1 if zero_init_state else 0, _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_scan_prefill_xproj(weights: ScanWeights, dims: Dims, u, conv_state, zero_init_state: bool,
+                              xdbl, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_scan_prefill_xproj", load().sambay_scan_prefill_xproj(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u), _p(conv_state), 1 if zero_init_state else 0,
+        _p(xdbl), _p(ws), ws_bytes, _stream(stream)))
+
+
+def sambay_scan_prefill_finish(weights: ScanWeights, dims: Dims, u, xdbl, M, ssm_state, conv_state,
+                               zero_init_state: bool, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sambay_scan_prefill_finish", load().sambay_scan_prefill_finish(
+        ctypes.byref(weights), ctypes.byref(dims), _p(u), _p(xdbl), _p(M), _p(ssm_state), _p(conv_state),
         1 if zero_init_state else 0, _p(ws), ws_bytes, _stream(stream)))
 
 
@@ -349,6 +373,18 @@ def gmu_forward(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=Non
     _check("gmu_forward", load().gmu_forward(
         ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(residual), _p(Y), _p(ws),
         ws_bytes, _stream(stream)))
+
+
+def gmu_forward_partial(dims: Dims, rows: int, X, M, W1, W2, Y_part, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("gmu_forward_partial", load().gmu_forward_partial(
+        ctypes.byref(dims), rows, _p(X), _p(M), _p(W1), _p(W2), _p(Y_part), _p(ws), ws_bytes,
+        _stream(stream)))
+
+
+def gmu_finish(dims: Dims, rows: int, Y_sum, residual, Y, stream=None):
+    _check("gmu_finish", load().gmu_finish(
+        ctypes.byref(dims), rows, _p(Y_sum), _p(residual), _p(Y), _stream(stream)))
 
 
 def gmu_step(dims: Dims, rows: int, X, M, W1, W2, residual, Y, ws, stream=None):

@@ -642,10 +642,19 @@ sambay::simt::Args simt_args(const float* A, long long sam, long long sak, const
 
 // ------------------------------------------------------------ shared scan pieces
 
+// Which part of the projections a call runs.  A channel-sharded prefill
+// stops after x_proj (PROJ_XPROJ: this shard's partial sums over its channels
+// into an external xdbl), the caller sums the partials over the shards, and
+// PROJ_FINISH takes the summed xdbl from there on.
+enum ProjPhase { PROJ_ALL, PROJ_XPROJ, PROJ_FINISH };
+
 // x_proj + dt_proj for `rows` tokens whose conv output is ws.uc:
 //   xdbl = uc W_x^T,  dt = softplus(delta W_dt^T + b_dt)
+// xdbl_ext: PROJ_XPROJ writes the (partial) xdbl there; PROJ_FINISH reads
+// the summed xdbl from there (and uc is not read).
 sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const sambay_dims* d,
-                          long long rows, uint8_t* ws, const ScanWs& L, cudaStream_t st, bool prefill) {
+                          long long rows, uint8_t* ws, const ScanWs& L, cudaStream_t st, bool prefill,
+                          ProjPhase phase = PROJ_ALL, float* xdbl_ext = nullptr) {
   const int Di = d->d_inner, R = d->dt_rank, ldx = d->dt_rank + 2 * d->d_state;
   float* xdbl = reinterpret_cast<float*>(ws + L.xdbl);
   float* dt = reinterpret_cast<float*>(ws + L.dt);
@@ -656,29 +665,40 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
     float* part = reinterpret_cast<float*>(ws + L.part);
     const long long stride = rows * ldx;
     const int Rp = rank_pad(R);
-    // x_proj = [uc_hi | uc_lo] [W_x | W_x]^T, split over K: each split writes
-    // its partial [rows, ldx] tile set
-    auto gx = tc_args(static_cast<int>(rows), ldx, 2 * Di, part, ldx, nullptr, nullptr, nullptr, stride);
-    gx.b_k_wrap = Di;
-    const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
-    constexpr int P = sambay::tc::EPI_F32_PARTIAL;
-    if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
-    else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
-    else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
-    else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+    if (phase != PROJ_FINISH) {
+      // x_proj = [uc_hi | uc_lo] [W_x | W_x]^T, split over K: each split writes
+      // its partial [rows, ldx] tile set
+      auto gx = tc_args(static_cast<int>(rows), ldx, 2 * Di, part, ldx, nullptr, nullptr, nullptr, stride);
+      gx.b_k_wrap = Di;
+      const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
+      constexpr int P = sambay::tc::EPI_F32_PARTIAL;
+      if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+      else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+      else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+      else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+    }
     {
+      // the split sums in a fixed order -> xdbl, the split delta and B | C
+      // pairs; PROJ_XPROJ: xdbl only (into xdbl_ext); PROJ_FINISH: the summed
+      // xdbl_ext is the single "split"
       auto k8 = sambay::scan::xdbl_reduce_kernel<8>;
       auto k1 = sambay::scan::xdbl_reduce_kernel<1>;
       SAMBAY_MAX_CARVEOUT(k8, dev);
       SAMBAY_MAX_CARVEOUT(k1, dev);
       const int Lseq = static_cast<int>(rows / d->batch), nrows = static_cast<int>(rows);
+      const float* src = phase == PROJ_FINISH ? xdbl_ext : part;
+      const int nsplit = phase == PROJ_FINISH ? 1 : L.splits;
+      float* dst = phase == PROJ_XPROJ ? xdbl_ext : xdbl;
+      bf16* dl = phase == PROJ_XPROJ ? nullptr : delta;
+      float* bp = phase == PROJ_XPROJ ? nullptr : bcp;
       ProfScope ps_reduce("xdbl_reduce", st);
-      const bool many = L.splits >= 16;
+      const bool many = nsplit >= 16;
       if (launch_k(many ? k8 : k1, dim3(grid_for(stride / 4 * (many ? 8 : 1), 256, sms)), dim3(256), 0, st, true, 1,
-                   part, L.splits, stride, xdbl, delta, bcp, Lseq, nrows, R, Rp, ldx) != cudaSuccess)
+                   src, nsplit, stride, dst, dl, bp, Lseq, nrows, R, Rp, ldx) != cudaSuccess)
         return SAMBAY_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
+    if (phase == PROJ_XPROJ) return SAMBAY_OK;
     // dt = softplus([delta_hi | delta_lo] [W_dt | W_dt]^T + b_dt); each half of
     // the A operand is padded with zeros to Rp, W_dt reads zeros past R
     auto gd = tc_args(static_cast<int>(rows), Di, 2 * Rp, dt, Di, nullptr, w->dt_bias);
@@ -690,18 +710,23 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
       SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_SOFTPLUS, false, 8>("dt_proj", dev, sms, a_d, b_wdt, gd, 1, st, true, true)));
   } else {
     const float* uc = reinterpret_cast<const float*>(ws + L.uc);
-    SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
-        simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
-                  ldx, Di, xdbl, ldx),
-        st));
+    if (phase != PROJ_FINISH) {
+      float* dst = phase == PROJ_XPROJ ? xdbl_ext : xdbl;
+      SAMBAY_TRY(run_simt<sambay::simt::F32_STORE>("x_proj_f32",
+          simt_args(uc, Di, 1, static_cast<const float*>(w->x_proj_w), 1, Di, static_cast<int>(rows),
+                    ldx, Di, dst, ldx),
+          st));
+      if (phase == PROJ_XPROJ) return SAMBAY_OK;
+    }
+    const float* xs = phase == PROJ_FINISH ? xdbl_ext : xdbl;
     if (prefill) {
       ProfScope ps_bc("bc_pairs", st);
       sambay::scan::bc_pairs_kernel<<<grid_for(rows * 2 * d->d_state, 256, 1 << 20), 256, 0, st>>>(
-          xdbl, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, ldx);
+          xs, bcp, static_cast<int>(rows / d->batch), static_cast<int>(rows), R, ldx);
       if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
     }
     SAMBAY_TRY(run_simt<sambay::simt::SOFTPLUS>("dt_proj_f32",
-        simt_args(xdbl, ldx, 1, static_cast<const float*>(w->dt_proj_w), 1, R,
+        simt_args(xs, ldx, 1, static_cast<const float*>(w->dt_proj_w), 1, R,
                   static_cast<int>(rows), Di, R, dt, Di, nullptr, w->dt_bias),
         st));
   }
@@ -752,11 +777,12 @@ sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cuda
 template <typename T>
 sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
                                 const sambay_dims* d, const void* u, void* M, float* ssm_state,
-                                void* conv_state, int zero_init, uint8_t* ws, cudaStream_t st) {
+                                void* conv_state, int zero_init, uint8_t* ws, cudaStream_t st,
+                                ProjPhase phase = PROJ_ALL, float* xdbl_ext = nullptr) {
   const long long T_ = static_cast<long long>(d->batch) * d->seqlen;
   const ScanWs L = scan_ws_layout(d, T_);
   T* uc = reinterpret_cast<T*>(ws + L.uc);
-  {
+  if (phase != PROJ_FINISH) {
     sambay::scan::ConvParams<T> p{static_cast<const T*>(u), static_cast<const T*>(conv_state),
                                   static_cast<const T*>(w->conv_w),
                                   static_cast<const T*>(w->conv_b), uc, d->batch, d->seqlen,
@@ -776,7 +802,8 @@ sambay_status scan_prefill_impl(int dev, int sms, const sambay_scan_weights* w,
     }
     if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
   }
-  SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st, true));
+  SAMBAY_TRY(projections(dev, sms, w, d, T_, ws, L, st, true, phase, xdbl_ext));
+  if (phase == PROJ_XPROJ) return SAMBAY_OK;
   {
     sambay::scan::ScanParams<T> p{};
     p.uc = uc;
@@ -938,6 +965,28 @@ sambay_status gmu_f32(const sambay_dims* d, long long rows, const void* X, const
                 static_cast<float*>(Y), Dm, static_cast<const float*>(residual)),
       st));
   return SAMBAY_OK;
+}
+
+// Y = io(Ysum + residual) over n elements (residual may be null); 4 per
+// thread (n is a multiple of 4: d_model is)
+template <typename T>
+__global__ void __launch_bounds__(256) gmu_finish_kernel(const float* __restrict__ Ysum,
+                                                         const T* __restrict__ residual, T* __restrict__ Y,
+                                                         long long n4) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 v = reinterpret_cast<const float4*>(Ysum)[i];
+    if (residual != nullptr) {
+      v.x += sambay::to_f32(residual[4 * i]);
+      v.y += sambay::to_f32(residual[4 * i + 1]);
+      v.z += sambay::to_f32(residual[4 * i + 2]);
+      v.w += sambay::to_f32(residual[4 * i + 3]);
+    }
+    Y[4 * i] = sambay::from_f32<T>(v.x);
+    Y[4 * i + 1] = sambay::from_f32<T>(v.y);
+    Y[4 * i + 2] = sambay::from_f32<T>(v.z);
+    Y[4 * i + 3] = sambay::from_f32<T>(v.w);
+  }
 }
 
 sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* X, const void* M,
@@ -1114,6 +1163,43 @@ sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const sambay_dim
   return scan_prefill_impl<float>(dev, sms, w, d, u, M, ssm_state, conv_state, zi, w8, st);
 }
 
+sambay_status sambay_scan_prefill_xproj(const sambay_scan_weights* w, const sambay_dims* d, const void* u,
+                                        const void* conv_state, int zero_init_state, float* xdbl, void* ws,
+                                        size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, false, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u, conv_state, xdbl}));
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_scan_prefill_workspace(d)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int zi = zero_init_state ? 1 : 0;
+  void* cs = const_cast<void*>(conv_state);   // read only in this phase
+  if (d->io == SAMBAY_BF16)
+    return scan_prefill_impl<bf16>(dev, sms, w, d, u, nullptr, nullptr, cs, zi, w8, st, PROJ_XPROJ, xdbl);
+  return scan_prefill_impl<float>(dev, sms, w, d, u, nullptr, nullptr, cs, zi, w8, st, PROJ_XPROJ, xdbl);
+}
+
+sambay_status sambay_scan_prefill_finish(const sambay_scan_weights* w, const sambay_dims* d, const void* u,
+                                         const float* xdbl, void* M, float* ssm_state, void* conv_state,
+                                         int zero_init_state, void* ws, size_t ws_bytes, sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, false, true));
+  SAMBAY_TRY(check_weights(w));
+  SAMBAY_TRY(check_ptrs({u, xdbl, M, ssm_state, conv_state}));
+  if (M == u) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ws(ws, ws_bytes, sambay_scan_prefill_workspace(d)));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int zi = zero_init_state ? 1 : 0;
+  float* xs = const_cast<float*>(xdbl);      // read only in this phase
+  if (d->io == SAMBAY_BF16)
+    return scan_prefill_impl<bf16>(dev, sms, w, d, u, M, ssm_state, conv_state, zi, w8, st, PROJ_FINISH, xs);
+  return scan_prefill_impl<float>(dev, sms, w, d, u, M, ssm_state, conv_state, zi, w8, st, PROJ_FINISH, xs);
+}
+
 sambay_status sambay_scan_step(const sambay_scan_weights* w, const sambay_dims* d, const void* u_t,
                                void* m_t, float* ssm_state, void* conv_state, void* ws,
                                size_t ws_bytes, sambay_stream_t stream) {
@@ -1157,6 +1243,53 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
       st, true, true, tail, L.tail_bytes, "gmu_out_tail")));
   return SAMBAY_OK;
+}
+
+sambay_status gmu_forward_partial(const sambay_dims* d, int64_t rows, const void* X, const void* M,
+                                  const void* W1, const void* W2, float* Y_part, void* ws, size_t ws_bytes,
+                                  sambay_stream_t stream) {
+  SAMBAY_TRY(gmu_common_checks(d, rows, X, M, W1, W2, nullptr, Y_part));
+  if (Y_part == X) return SAMBAY_ERR_INVALID_ARG;
+  const GmuWs L = gmu_ws_layout(d, rows, false);
+  SAMBAY_TRY(check_ws(ws, ws_bytes, L.total));
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  if (d->io == SAMBAY_F32) return gmu_f32(d, rows, X, M, W1, W2, nullptr, Y_part, w8, L, st);
+  const int Dm = d->d_model, Di = d->d_inner, T = static_cast<int>(rows);
+  bf16* H = reinterpret_cast<bf16*>(w8 + L.h);
+  float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
+  SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 4, true>(
+      "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, false,
+      true, tail, L.tail_bytes, "gmu_gate_tail")));
+  // Y_part = H W2 in fp32: single-CTA 128 x 256 tiles (the CTA-pair form has
+  // only the bf16 epilogues), whole tiles only
+  SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_F32_PARTIAL, false, 4>(
+      "gmu_out_partial", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y_part, Dm), 1, st,
+      true, false)));
+  return SAMBAY_OK;
+}
+
+sambay_status gmu_finish(const sambay_dims* d, int64_t rows, const float* Y_sum, const void* residual, void* Y,
+                         sambay_stream_t stream) {
+  SAMBAY_TRY(check_dims(d, true, false));
+  if (rows < 1 || rows > (1LL << 30)) return SAMBAY_ERR_INVALID_ARG;
+  SAMBAY_TRY(check_ptrs({Y_sum, Y}));
+  if (residual && !aligned16(residual)) return SAMBAY_ERR_UNSUPPORTED;
+  if (Y == static_cast<const void*>(Y_sum)) return SAMBAY_ERR_INVALID_ARG;
+  int dev, sms;
+  SAMBAY_TRY(current_device(&dev, &sms));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long n4 = rows * d->d_model / 4;
+  ProfScope ps("gmu_finish", st);
+  if (d->io == SAMBAY_BF16)
+    gmu_finish_kernel<bf16><<<grid_for(n4, 256, sms), 256, 0, st>>>(Y_sum, static_cast<const bf16*>(residual),
+                                                                    static_cast<bf16*>(Y), n4);
+  else
+    gmu_finish_kernel<float><<<grid_for(n4, 256, sms), 256, 0, st>>>(Y_sum, static_cast<const float*>(residual),
+                                                                     static_cast<float*>(Y), n4);
+  return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
 }
 
 sambay_status gmu_step(const sambay_dims* d, int64_t rows, const void* X, const void* M,

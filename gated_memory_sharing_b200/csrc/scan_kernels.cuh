@@ -186,7 +186,8 @@ __global__ void __launch_bounds__(CB / 4 * (kConvTT / 4), 4) conv_silu_kernel(co
 // result does not depend on scheduling.  The delta columns are also written
 // as the split bf16 A operand of the dt_proj GEMM: delta2 [rows, 2*Rp] with
 // hi in columns [0, R), lo in [Rp, Rp + R) and zeros in the padding up to
-// Rp (a multiple of 64).  One thread: 4 consecutive columns.
+// Rp (a multiple of 64).  One thread: 4 consecutive columns.  delta2 and bcp
+// may be null: xdbl only.
 
 // LPG lanes per 4-column group: lane `sub` adds splits sub, sub + LPG, ... in
 // order, then a fixed xor tree combines the lane sums, so the result is the
@@ -239,6 +240,7 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
     const long long row = e / ldx;
     const int col = static_cast<int>(e % ldx);
     if (col < R) {
+      if (delta2 == nullptr) continue;   // xdbl only (a shard's partial sums)
       const float a[4] = {acc.x, acc.y, acc.z, acc.w};
       bf16 hi[4], lo[4];
 #pragma unroll
@@ -266,6 +268,7 @@ __global__ void xdbl_reduce_kernel(const float* __restrict__ partials, int split
     }
   }
   // zero padding columns [R, Rp) of both halves
+  if (delta2 == nullptr) return;
   const int pad4 = (Rp - R) / 4;
   const long long totalp = static_cast<long long>(rows) * pad4 * 2;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < totalp;

@@ -138,6 +138,39 @@ SAMBAY_API sambay_status sambay_scan_prefill(const sambay_scan_weights* w, const
                                   sambay_stream_t stream);
 
 /*
+ * Channel-sharded prefill (one shard of d_inner per GPU).  The scan is
+ * independent per channel except for x_proj, whose [delta | B | C] sums run
+ * over all channels [MAMBA] (selection projections), so sambay_scan_prefill
+ * splits there into two calls around the caller's sum over the shards (an
+ * all-reduce of xdbl):
+ *
+ * sambay_scan_prefill_xproj - conv + SiLU and this shard's x_proj partial
+ * sums.  dims->d_inner and the weights are the shard's (conv_w, conv_b,
+ * x_proj_w [R + 2N, Di_shard], dt_proj_w [Di_shard, R], dt_bias, A, D of its
+ * channels); u [B, L, Di_shard] io is its slice of the scan input.
+ *   conv_state  [B, Di_shard, K] io  in (read only here; the left context
+ *               unless zero_init_state).
+ *   xdbl        [B*L, R + 2N] f32 out: sum over the shard's channels of
+ *               uc * W_x^T (deterministic order).  Caller-owned, 16-byte
+ *               aligned.
+ *   ws          >= sambay_scan_prefill_workspace(dims); it carries the conv
+ *               output to the second call and must be passed there unchanged.
+ * sambay_scan_prefill_finish - given xdbl summed over all shards: delta, B,
+ * C, dt_proj + softplus and the scan of the shard's channels; writes M
+ * [B, L, Di_shard] and updates ssm_state / conv_state exactly as
+ * sambay_scan_prefill does.  u, conv_state, zero_init_state and ws as in the
+ * first call.  With one shard the pair computes what sambay_scan_prefill
+ * computes.
+ */
+SAMBAY_API sambay_status sambay_scan_prefill_xproj(const sambay_scan_weights* w, const sambay_dims* dims,
+                                        const void* u, const void* conv_state, int zero_init_state,
+                                        float* xdbl, void* ws, size_t ws_bytes, sambay_stream_t stream);
+SAMBAY_API sambay_status sambay_scan_prefill_finish(const sambay_scan_weights* w, const sambay_dims* dims,
+                                         const void* u, const float* xdbl, void* M, float* ssm_state,
+                                         void* conv_state, int zero_init_state, void* ws,
+                                         size_t ws_bytes, sambay_stream_t stream);
+
+/*
  * sambay_scan_step - one decode token per sequence: the prefill with L = 1
  * on the carried state, updating ssm_state and conv_state IN PLACE [GMU]
  * (constant-size state), [MAMBA].  dims->seqlen is ignored.  In SAMBAY_BF16
@@ -184,6 +217,23 @@ SAMBAY_API sambay_status sambay_scan_step(const sambay_scan_weights* w, const sa
 SAMBAY_API sambay_status gmu_forward(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
                           const void* W1, const void* W2, const void* residual, void* Y,
                           void* ws, size_t ws_bytes, sambay_stream_t stream);
+
+/*
+ * gmu_forward_partial - the GMU of one d_inner shard [GMU]: H = M ⊙ SiLU(X
+ * W1^T) over the shard's channels (W1 [Di_shard, Dm], M [rows, Di_shard]),
+ * then Y_part = H W2 (W2 [Di_shard, Dm], the shard's rows) as float32
+ * [rows, Dm], with no residual.  The sum of Y_part over the shards (an
+ * all-reduce) is Y before the residual; gmu_finish completes it.  ws:
+ * >= gmu_forward_workspace(dims, rows) (dims->d_inner = the shard's).
+ *
+ * gmu_finish - Y = io(Y_sum + residual) (residual [rows, Dm] io or NULL;
+ * Y [rows, Dm] io, may alias residual, not Y_sum).
+ */
+SAMBAY_API sambay_status gmu_forward_partial(const sambay_dims* dims, int64_t rows, const void* X,
+                                  const void* M, const void* W1, const void* W2, float* Y_part,
+                                  void* ws, size_t ws_bytes, sambay_stream_t stream);
+SAMBAY_API sambay_status gmu_finish(const sambay_dims* dims, int64_t rows, const float* Y_sum,
+                         const void* residual, void* Y, sambay_stream_t stream);
 
 /*
  * gmu_step - the GMU for one decode token of `rows` sequences (rows <= 256)

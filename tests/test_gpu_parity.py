@@ -159,6 +159,24 @@ def test_scan_prefill_short_and_ragged(L):
     np.testing.assert_array_equal(host(cs), r["conv_state"])
 
 
+@pytest.mark.parametrize("B,L,Di,R", [
+    (2, 150, 320, 72),    # 300 tokens: 4 whole 64-token tiles + 44; 2.5 channel tiles; R < its 128 pad
+    (1, 129, 192, 160),   # one token past a tile; R = 160 padded to 192
+])
+def test_scan_prefill_ragged_projection_tiles(B, L, Di, R):
+    """Prefill whose dt projection has ragged token, channel and rank tiles."""
+    d = synth.Dims(B, L, 128, Di, 16, 4, R, synth.BF16)
+    seed = 25 + L + R
+    w = synth.scan_weights(d, seed)
+    u = synth.scan_inputs(d, seed)
+    layer = ScanLayer(w, d.d_model, abi.BF16)
+    M, h, cs = layer.prefill(to_device(u, abi.BF16))
+    r = ref.scan_prefill_ref(u, w)
+    assert_close(host(M), r["M"], TOL_BF16, f"scan B{B} L{L} Di{Di} R{R}")
+    assert_close(host(h), r["ssm_state"], TOL_BF16, "state")
+    np.testing.assert_array_equal(host(cs), r["conv_state"])
+
+
 @pytest.mark.parametrize("name", ["f32", "bf16"])
 def test_scan_prefill_continues_state(name):
     d = SMALL[name]
