@@ -352,13 +352,19 @@ __host__ __device__ constexpr int uc_parts() { return sizeof(T) == 2 ? 2 : 1; }
 template <typename T>
 __device__ __forceinline__ long long uc_ld(int Di) { return static_cast<long long>(Di) * uc_parts<T>(); }
 
-// Dynamic shared memory of one CTA.  Rows of the channel tiles are `pitch`
-// elements, pitch = 4 (mod 32): a warp's 8-token x 4-channel preload then
-// touches 32 distinct banks.
+// Dynamic shared memory of one CTA.  Rows of the channel tiles are
+// kScanPitch = 36 elements (at least the kScanMaxCH channels of any CTA, and
+// 4 mod 32: a warp's 8-token x 4-channel preload then touches 32 distinct
+// banks).  A compile-time pitch lets the chunk loop address its tiles with
+// immediate offsets.
+constexpr int kScanPitch = 36;
+static_assert(kScanPitch >= kScanMaxCH && kScanPitch % 32 == 4, "scan tile pitch");
+
 struct ScanLayout {
   int pitch, dt, uc, bc, out, bytes;
   __host__ __device__ ScanLayout(int chp, int tsize) {
-    pitch = chp + (36 - chp % 32) % 32;
+    (void)chp;
+    pitch = kScanPitch;
     const int parts = tsize == 2 ? 2 : 1;
     dt = 0;
     uc = dt + kScanStages * kScanTC * pitch * 4;
@@ -500,7 +506,7 @@ __global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(cons
   extern __shared__ __align__(16) uint8_t scan_smem_raw[];
   uint8_t* smem = scan_smem_raw;
   const ScanLayout ly(p.chp, sizeof(T));
-  const int pitch = ly.pitch;
+  constexpr int pitch = kScanPitch;
   const int blk = blockIdx.x, b = blockIdx.y;
   const int CH = 4 * (p.q_base + (blk < p.q_extra ? 1 : 0));
   const int c0 = 4 * (blk * p.q_base + min(blk, p.q_extra));
@@ -509,8 +515,11 @@ __global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(cons
   const int lane = threadIdx.x & 31;
   const int cl = (threadIdx.x >> 5) * 4 + (lane & 3), q = lane >> 2;
   const bool active = cl < CH;
-  const int col = active ? cl : 0;               // lanes past CH shadow channel 0
-  const int c = c0 + col;
+  // lanes past CH (a CTA narrower than chp) read their global parameters as
+  // channel c0 and run on the tile columns [CH, chp), which no copy fills or
+  // empties: their results stay in staging columns that never reach M
+  const int col = cl;
+  const int c = c0 + (active ? cl : 0);
   const float a2_0 = p.A[static_cast<long long>(c) * kN + 2 * q] * kLog2e;
   const float a2_1 = p.A[static_cast<long long>(c) * kN + 2 * q + 1] * kLog2e;
   float* hp = p.h + (static_cast<long long>(b) * p.Di + c) * kN + 2 * q;
@@ -548,7 +557,7 @@ __global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(cons
     const float* dtc = s_dt + st * kScanTC * pitch + col;
     const T* ucc = s_uc + st * uc_parts<T>() * kScanTC * pitch + col;
     const float4* bcc = s_bc + st * (kScanTC / 2) * 16 + q;
-#pragma unroll 2
+#pragma unroll
     for (int g = 0; g < kScanTC; g += 8) {
       // this lane's token g+q: dt, uc, dt*uc
       const int tq = g + q;
@@ -580,7 +589,7 @@ __global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(cons
         v[i + 1] = pr2.y;
       }
       const float y = fmaf(Dc, uq, reduce_scatter8(v, q));
-      if (active) s_out[(ob * kScanTC + tq) * pitch + col] = from_f32<T>(y);
+      s_out[(ob * kScanTC + tq) * pitch + col] = from_f32<T>(y);
     }
   }
   __syncthreads();
