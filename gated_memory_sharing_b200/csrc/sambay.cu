@@ -589,8 +589,17 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
     const long long work = static_cast<long long>(ktail) * C::kBMT * (BN / 4) * kTailLanes;
     auto rk = tail_reduce_kernel<BN, C::kBMT, KIND>;
     SAMBAY_MAX_CARVEOUT(rk, dev);
+    // one resident wave (the grid-stride loop takes the rest): a second wave
+    // would pay the partials' L2 round trip again
+    static int per_sm[kMaxDevices] = {};
+    if (per_sm[dev] == 0) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rk, 256, 0) != cudaSuccess || n < 1) n = 1;
+      per_sm[dev] = n;
+    }
+    const int grid = static_cast<int>(std::min<long long>((work + 255) / 256, static_cast<long long>(per_sm[dev]) * sms));
     ProfScope ps(tail_name ? tail_name : "gemm_tail_reduce", st);
-    if (launch_k(rk, dim3(grid_for(work, 256, sms)), dim3(256), 0, st, true, 1, g, ktail) != cudaSuccess)
+    if (launch_k(rk, dim3(grid), dim3(256), 0, st, true, 1, g, ktail) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;

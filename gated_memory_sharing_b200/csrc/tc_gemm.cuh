@@ -1263,6 +1263,14 @@ __global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmArgs g, int 
     const int n = (tile / g.m_tiles) * BN + 4 * lq;
     const bool live = e < total && m < g.M && n < g.N;
     const float* base = g.tail_part + (static_cast<long long>(i) * g.tail_ksplit * BMT + lr) * BN + 4 * lq;
+    const long long o = static_cast<long long>(m) * g.ldo + n;
+    // the aux (M or the residual) of the reducing lane's 4 outputs, loaded
+    // together with the partials so the two round trips overlap
+    constexpr bool kAuxKind = KIND == EPI_GATE || KIND == EPI_RESID;
+    const bool vec4 = n + 4 <= g.N && (o & 3) == 0;
+    uint2 aux4 = make_uint2(0u, 0u);
+    if (kAuxKind && g.aux != nullptr && live && sub == 0 && vec4)
+      aux4 = __ldcg(reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(g.aux) + o));
     float4 x[PER];
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
@@ -1284,7 +1292,20 @@ __global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmArgs g, int 
     }
     if (!live || sub != 0) continue;
     const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-    const long long o = static_cast<long long>(m) * g.ldo + n;
+    if (kAuxKind && vec4) {
+      // 4 bf16 outputs as one 8-byte store
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&aux4);
+      const float2 a01 = __bfloat1622float2(a2[0]), a23 = __bfloat1622float2(a2[1]);
+      const float a[4] = {a01.x, a01.y, a23.x, a23.y};
+      float r[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r[j] = KIND == EPI_GATE ? silu(v[j]) * a[j] : v[j] + a[j];
+      uint2 packed;
+      *reinterpret_cast<__nv_bfloat162*>(&packed.x) = __floats2bfloat162_rn(r[0], r[1]);
+      *reinterpret_cast<__nv_bfloat162*>(&packed.y) = __floats2bfloat162_rn(r[2], r[3]);
+      *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(g.out) + o) = packed;
+      continue;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (n + j >= g.N) break;
