@@ -767,10 +767,16 @@ template <typename T>
 sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cudaStream_t st) {
   using namespace sambay::scan;
   auto kern = selective_scan_kernel<T>;
+  // Two CTAs fit on an SM (registers and shared memory), which hides more of
+  // the recurrence's latency when the grid has more CTAs than SMs.  A grid of
+  // at most one CTA per SM asks for more than half an SM's shared memory
+  // instead, so that, launched early behind the kernel before it, its CTAs
+  // cannot pair up on the SMs that free first while others stay empty.
+  constexpr int kSoloSmem = 120 * 1024;
   static bool attr_set[kMaxDevices] = {};
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ScanLayout(kScanMaxCH, sizeof(T)).bytes) != cudaSuccess)
+                             std::max(ScanLayout(kScanMaxCH, sizeof(T)).bytes, kSoloSmem)) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
     attr_set[dev] = true;
   }
@@ -778,9 +784,11 @@ sambay_status launch_scan(int dev, int sms, sambay::scan::ScanParams<T>& p, cuda
   scan_partition<T>(p, sms);
   const ScanLayout ly(p.chp, sizeof(T));
   dim3 grid(p.nblk, p.B);
+  const bool solo = static_cast<long long>(p.nblk) * p.B <= sms;
+  const size_t smem = solo ? std::max(ly.bytes, kSoloSmem) : static_cast<size_t>(ly.bytes);
   ProfScope ps("selective_scan", st);
-  return launch_k(kern, grid, dim3(8 * p.chp), ly.bytes, st, true, 1, p) == cudaSuccess ? SAMBAY_OK
-                                                                        : SAMBAY_ERR_CUDA;
+  return launch_k(kern, grid, dim3(8 * p.chp), smem, st, true, 1, p) == cudaSuccess ? SAMBAY_OK
+                                                                   : SAMBAY_ERR_CUDA;
 }
 
 template <typename T>

@@ -500,7 +500,7 @@ __device__ __forceinline__ void scan_write_piece(const ScanParams<T>& p, const T
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kScanMaxThreads, 1) selective_scan_kernel(const ScanParams<T> p) {
+__global__ void __launch_bounds__(kScanMaxThreads, 2) selective_scan_kernel(const ScanParams<T> p) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t scan_smem_raw[];
