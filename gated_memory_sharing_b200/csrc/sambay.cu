@@ -681,7 +681,11 @@ sambay_status projections(int dev, int sms, const sambay_scan_weights* w, const 
       gx.b_k_wrap = Di;
       const Operand a_uc{uc, rows, 2LL * Di}, b_wx{w->x_proj_w, ldx, Di};
       constexpr int P = sambay::tc::EPI_F32_PARTIAL;
-      if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+      if (rows > 256 && ldx > 128 && ldx <= 192) {
+        // prefill: 256-row tiles on CTA pairs, each CTA loading half of the
+        // W_x tile (the splits' K ranges as in the single-CTA form)
+        SAMBAY_TRY((run_tc<192, false, false, P, false, 4, true>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
+      } else if (ldx <= 64) SAMBAY_TRY((run_tc<64, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
       else if (ldx <= 128) SAMBAY_TRY((run_tc<128, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
       else if (ldx <= 192) SAMBAY_TRY((run_tc<192, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));
       else SAMBAY_TRY((run_tc<256, false, false, P, false>("x_proj", dev, sms, a_uc, b_wx, gx, L.splits, st, true)));

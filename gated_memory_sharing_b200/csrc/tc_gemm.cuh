@@ -532,7 +532,7 @@ struct Cfg {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, whole 32-column epilogue chunks");
   static_assert(!TRANS || EW == 4, "decode epilogue: one warp per TMEM lane quarter");
   static_assert(!B_MN || kBHalf % 64 == 0, "MN-major B tiles are whole 64-element atoms");
-  static_assert(!PAIR || (!TRANS && !A_MN && KIND != EPI_F32_PARTIAL), "pairs serve the row-major prefill GEMMs");
+  static_assert(!PAIR || (!TRANS && !A_MN), "pairs serve the row-major prefill GEMMs");
 };
 
 struct TileCoord {

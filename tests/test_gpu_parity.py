@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from gated_memory_sharing_b200 import abi, synth
-from gated_memory_sharing_b200.layers import GMULayer, ScanLayer, to_device
+from gated_memory_sharing_b200.layers import GMULayer, ScanLayer, to_device, to_device_f32
 from oracle import sambay_ref as ref
 from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, host
 
@@ -162,9 +162,11 @@ def test_scan_prefill_short_and_ragged(L):
 @pytest.mark.parametrize("B,L,Di,R", [
     (2, 150, 320, 72),    # 300 tokens: 4 whole 64-token tiles + 44; 2.5 channel tiles; R < its 128 pad
     (1, 129, 192, 160),   # one token past a tile; R = 160 padded to 192
+    (2, 200, 256, 128),   # x_proj (R + 32 = 160 columns) on CTA pairs: a 256-row tile and a 144-row one
 ])
 def test_scan_prefill_ragged_projection_tiles(B, L, Di, R):
-    """Prefill whose dt projection has ragged token, channel and rank tiles."""
+    """Prefill whose x_proj / dt projection tiles are ragged in tokens,
+    channels and rank."""
     d = synth.Dims(B, L, 128, Di, 16, 4, R, synth.BF16)
     seed = 25 + L + R
     w = synth.scan_weights(d, seed)
@@ -174,6 +176,29 @@ def test_scan_prefill_ragged_projection_tiles(B, L, Di, R):
     r = ref.scan_prefill_ref(u, w)
     assert_close(host(M), r["M"], TOL_BF16, f"scan B{B} L{L} Di{Di} R{R}")
     assert_close(host(h), r["ssm_state"], TOL_BF16, "state")
+    np.testing.assert_array_equal(host(cs), r["conv_state"])
+
+
+@pytest.mark.parametrize("io", [synth.BF16, synth.F32])
+def test_scan_prefill_wide_warp_quads(io):
+    """8 sequences x 640 channels: the partition makes 18 CTAs per sequence,
+    16 of nine quads (the ninth on the two 16-lanes-per-channel warps) and 2
+    of eight, over 70 tokens (a ragged third chunk), from a given state."""
+    d = synth.Dims(8, 70, 128, 640, 16, 4, 16, io)
+    aio, tol = _io(io)
+    seed = 29
+    w = synth.scan_weights(d, seed)
+    u = synth.scan_inputs(d, seed)
+    rng = np.random.default_rng(3)
+    h0 = rng.standard_normal((d.batch, d.d_inner, 16)).astype(np.float32)
+    cs0 = synth.round_bf16(rng.standard_normal((d.batch, d.d_inner, 4)).astype(np.float32)) \
+        if io == synth.BF16 else rng.standard_normal((d.batch, d.d_inner, 4)).astype(np.float32)
+    layer = ScanLayer(w, d.d_model, aio)
+    h, cs = to_device_f32(h0), to_device(cs0, aio)
+    M, h, cs = layer.prefill(to_device(u, aio), h, cs, fresh=False)
+    r = ref.scan_prefill_ref(u, w, h0, cs0)
+    assert_close(host(M), r["M"], tol, f"scan M wide quads {io}")
+    assert_close(host(h), r["ssm_state"], tol, "state")
     np.testing.assert_array_equal(host(cs), r["conv_state"])
 
 
