@@ -180,10 +180,11 @@ def test_scan_prefill_ragged_projection_tiles(B, L, Di, R):
 
 
 @pytest.mark.parametrize("io", [synth.BF16, synth.F32])
-def test_scan_prefill_wide_warp_quads(io):
+def test_scan_prefill_mixed_cta_widths(io):
     """8 sequences x 640 channels: the partition makes 18 CTAs per sequence,
-    16 of nine quads (the ninth on the two 16-lanes-per-channel warps) and 2
-    of eight, over 70 tokens (a ragged third chunk), from a given state."""
+    16 of nine 4-channel quads and 2 of eight (the narrower CTAs' spare lanes
+    run on unused tile columns), over 70 tokens (a ragged third chunk), from
+    a given state."""
     d = synth.Dims(8, 70, 128, 640, 16, 4, 16, io)
     aio, tol = _io(io)
     seed = 29
@@ -197,7 +198,7 @@ def test_scan_prefill_wide_warp_quads(io):
     h, cs = to_device_f32(h0), to_device(cs0, aio)
     M, h, cs = layer.prefill(to_device(u, aio), h, cs, fresh=False)
     r = ref.scan_prefill_ref(u, w, h0, cs0)
-    assert_close(host(M), r["M"], tol, f"scan M wide quads {io}")
+    assert_close(host(M), r["M"], tol, f"scan M mixed CTA widths {io}")
     assert_close(host(h), r["ssm_state"], tol, "state")
     np.testing.assert_array_equal(host(cs), r["conv_state"])
 
