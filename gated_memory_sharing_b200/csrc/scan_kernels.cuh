@@ -102,6 +102,27 @@ __device__ __forceinline__ void store_uc(T* uc, long long row, int Di, int c0, c
   }
 }
 
+// 4 conv outputs at `dst` (a row of uc, column c): float32 as is; bf16 as
+// the split pair, hi at dst and lo Di elements further
+template <typename T>
+__device__ __forceinline__ void store_uc_row(T* dst, int Di, const float (&y)[4]) {
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]), h1 = __floats2bfloat162_rn(y[2], y[3]);
+    const float2 b0 = __bfloat1622float2(h0), b1 = __bfloat1622float2(h1);
+    const __nv_bfloat162 l0 = __floats2bfloat162_rn(y[0] - b0.x, y[1] - b0.y);
+    const __nv_bfloat162 l1 = __floats2bfloat162_rn(y[2] - b1.x, y[3] - b1.y);
+    uint2 hi, lo;
+    hi.x = *reinterpret_cast<const uint32_t*>(&h0);
+    hi.y = *reinterpret_cast<const uint32_t*>(&h1);
+    lo.x = *reinterpret_cast<const uint32_t*>(&l0);
+    lo.y = *reinterpret_cast<const uint32_t*>(&l1);
+    *reinterpret_cast<uint2*>(dst) = hi;
+    *reinterpret_cast<uint2*>(dst + Di) = lo;
+  } else {
+    *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
+  }
+}
+
 // 4 consecutive values of T at p (8- or 16-byte aligned) as floats
 template <typename T>
 __device__ __forceinline__ void load4(const T* p, float (&x)[4]) {
@@ -161,22 +182,25 @@ __global__ void __launch_bounds__(CB / 4 * (kConvTT / 4), 4) conv_silu_kernel(co
   __syncthreads();
 
   // output token t0 + 4tq + i reads tile rows 4tq + i .. 4tq + i + K - 1
-  // (tile row r is token t0 - K + 1 + r)
+  // (tile row r is token t0 - K + 1 + r): the thread's 4 + K - 1 rows are
+  // read and converted once, and its output rows are one pointer step apart
+  float x[4 + kK - 1][4];
+#pragma unroll
+  for (int r = 0; r < 4 + kK - 1; ++r) load4<T>(&tile[4 * tq + r][4 * j], x[r]);
+  const long long ld = static_cast<long long>(p.Di) * (sizeof(T) == 2 ? 2 : 1);   // uc row: split pair or f32
+  T* dst = p.uc + (base + t0 + 4 * tq) * ld + cj;
+  const int nt = min(4, p.L - (t0 + 4 * tq));
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int t = t0 + 4 * tq + i;
-    if (t >= p.L) break;
+    if (i >= nt) break;
     float y[4] = {bias[0], bias[1], bias[2], bias[3]};
 #pragma unroll
-    for (int k = 0; k < kK; ++k) {
-      float x[4];
-      load4<T>(&tile[4 * tq + i + k][4 * j], x);
+    for (int k = 0; k < kK; ++k)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) y[v] = fmaf(w[v][k], x[v], y[v]);
-    }
+      for (int v = 0; v < 4; ++v) y[v] = fmaf(w[v][k], x[i + k][v], y[v]);
 #pragma unroll
     for (int v = 0; v < 4; ++v) y[v] = silu(y[v]);
-    store_uc<T, 4>(p.uc, base + t, p.Di, cj, y);
+    store_uc_row<T>(dst + i * ld, p.Di, y);
   }
 }
 
