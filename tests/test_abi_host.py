@@ -305,3 +305,35 @@ def test_ssd_argument_errors(lib):
         abi.sambay_ssd_prefill(w, ok, p, _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000),
                                _FakePtr(0x50000), True, p, 0)
     assert e.value.code == 3
+
+
+def test_sharded_prefill_argument_errors(lib):
+    """The channel-sharded prefill's calls reject bad arguments on the host,
+    before any launch (status codes 1 invalid, 2 unsupported, 3 workspace)."""
+    ok = abi.make_dims(1, 64, 128, 256, 16, 4, 16, abi.BF16)
+    w = abi.ScanWeights(*([0x10000] * 7))
+    u, cs, M, h = _FakePtr(0x20000), _FakePtr(0x30000), _FakePtr(0x40000), _FakePtr(0x50000)
+    big_ws = _FakePtr(0x60000)
+    big_ws.numel = lambda: abi.sambay_scan_prefill_workspace(ok)
+    cases = [
+        (lambda: abi.sambay_scan_prefill_xproj(w, ok, u, cs, True, None, big_ws, 0), 1),              # no xdbl
+        (lambda: abi.sambay_scan_prefill_xproj(w, ok, u, cs, True, _FakePtr(0x70004), big_ws, 0), 2),  # misaligned
+        (lambda: abi.sambay_scan_prefill_xproj(w, ok, u, cs, True, _FakePtr(0x70000), _FakePtr(0x60000), 0), 3),
+        (lambda: abi.sambay_scan_prefill_xproj(w, abi.make_dims(1, 64, 128, 256, 32, 4, 16, abi.BF16), u, cs,
+                                               True, _FakePtr(0x70000), big_ws, 0), 2),                # d_state
+        (lambda: abi.sambay_scan_prefill_finish(w, ok, u, _FakePtr(0x70000), u, h, cs, True, big_ws, 0), 1),  # M is u
+        (lambda: abi.sambay_scan_prefill_finish(w, ok, u, None, M, h, cs, True, big_ws, 0), 1),        # no xdbl
+    ]
+    g = abi.make_dims(64, 1, 128, 256, 16, 4, 4, abi.BF16)
+    X, Mg, W1, W2, Yp = (_FakePtr(a) for a in (0x20000, 0x30000, 0x40000, 0x50000, 0x60000))
+    cases += [
+        (lambda: abi.gmu_forward_partial(g, 0, X, Mg, W1, W2, Yp, big_ws, 0), 1),                      # no rows
+        (lambda: abi.gmu_forward_partial(g, 64, X, Mg, W1, W2, X, big_ws, 0), 1),                      # Y_part is X
+        (lambda: abi.gmu_finish(g, 0, Yp, None, X, 0), 1),                                             # no rows
+        (lambda: abi.gmu_finish(g, 64, Yp, None, Yp, 0), 1),                                           # Y is Y_sum
+        (lambda: abi.gmu_finish(g, 64, Yp, _FakePtr(0x70002), X, 0), 2),                               # residual
+    ]
+    for call, code in cases:
+        with pytest.raises(abi.SambayError) as e:
+            call()
+        assert e.value.code == code
