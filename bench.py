@@ -20,6 +20,13 @@ method are measured in the same run and reported under "workloads":
                            34816 cached tokens: the 2K prompt and the end of
                            32K generated ones) and through a GMU layer: bytes
                            and time per decoded token of each
+  sambay2_prefill_b1_l2048 the SambaY-2 memory readout (Mamba-2 SSD scan) of
+                           a 2048-token prompt, 80 heads of 64, d_state 128
+  mamba_layer_b1_l2048     the whole Mamba layer from X at the headline sizes:
+                           in_proj, the scan, (y ⊙ SiLU(X W_z^T)) W_out + X
+  sambay_mlp_b1_l2048      SambaY-MLP at the headline sizes: the SwiGLU hidden
+                           activation of X_self as the memory of a GMU layer
+                           gated by X_cross
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--only-headline] [--no-cpu-baseline]
@@ -48,8 +55,9 @@ sys.path.insert(0, ROOT)
 from gated_memory_sharing_b200 import synth  # noqa: E402
 
 HEADLINE = "prefill_b1_l2048"
+LAYER_WORKLOADS = ("mamba_layer_b1_l2048", "sambay_mlp_b1_l2048")
 WORKLOADS = ("prefill_b1_l2048", "decode_b64", "long_prefill_b4_l32768", "sharing_b2_l8192",
-             "sharing_decode_b16", "cross_attn_vs_gmu_b64", "sambay2_prefill_b1_l2048")
+             "sharing_decode_b16", "cross_attn_vs_gmu_b64", "sambay2_prefill_b1_l2048") + LAYER_WORKLOADS
 UNIT = "tokens/s"
 METRICS = {
     "prefill_b1_l2048": "scan+GMU prefill tokens/s",
@@ -59,6 +67,8 @@ METRICS = {
     "sharing_decode_b16": "scan+8xGMU decode tokens/s",
     "cross_attn_vs_gmu_b64": "cross-attention decode tokens/s at 2048 cached tokens",
     "sambay2_prefill_b1_l2048": "SambaY-2 (Mamba-2 SSD) memory readout prefill tokens/s",
+    "mamba_layer_b1_l2048": "Mamba layer (in_proj + scan + gated out_proj) prefill tokens/s",
+    "sambay_mlp_b1_l2048": "SambaY-MLP memory (SwiGLU hidden activation) + GMU prefill tokens/s",
 }
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch, from an
 # earlier ncu capture of the headline workload, for kernels unchanged since
@@ -214,6 +224,9 @@ def dev_normal(shape, seed, device):
 
 def workload_dims(name):
     """(dims, seed, gmu layers, decode?) of a bench workload."""
+    if name in LAYER_WORKLOADS:
+        d, seed = synth.workload(HEADLINE)
+        return d, seed, 1, False
     if name == "sambay2_prefill_b1_l2048":
         return synth.SSD_WORKLOAD, synth.SSD_WORKLOAD_SEED, 0, False
     if name == "cross_attn_vs_gmu_b64":
@@ -237,6 +250,12 @@ def config_of(name, d, layers, decode):
     c = {"workload": name, "batch": d.batch, "seq_len": d.seqlen, "d_model": d.d_model,
          "d_inner": d.d_inner, "d_state": d.d_state, "d_conv": d.d_conv, "dt_rank": d.dt_rank,
          "gmu_layers": layers}
+    if name == "mamba_layer_b1_l2048":
+        c.pop("gmu_layers")
+        c["layer"] = "in_proj (x branch) + scan + gated out_proj + residual"
+    if name == "sambay_mlp_b1_l2048":
+        c = {"workload": name, "batch": d.batch, "seq_len": d.seqlen, "d_model": d.d_model, "d_ff": d.d_inner,
+             "gmu_layers": 1}
     if decode:
         c["prompt"] = d.seqlen
         c.pop("seq_len")
@@ -287,6 +306,25 @@ def cpu_baseline(name, budget_s=8.0, reps_max=4):
         return {"value": reps * S / el, "unit": UNIT, "cores": cores, "kind": "oracle",
                 "sample": f"cross-attention decode of {S} sequences over {N} cached tokens x {reps}, "
                           f"{el:.1f} s of float64 NumPy"}
+    if name in LAYER_WORKLOADS:
+        L = 256
+        X = synth.gmu_inputs(d, seed, rows=L)
+        reps, t0 = 0, time.perf_counter()
+        if name == "mamba_layer_b1_l2048":
+            w, bw = synth.scan_weights(d, seed), synth.mamba_block_weights(d, seed)
+            run = lambda: ref.mamba_layer_ref(X[None], w, bw["W_in"], bw["W_z"], bw["W_out"])
+            what = "in_proj + scan + gated out_proj"
+        else:
+            mw, gw = synth.mlp_weights(d, seed), synth.gmu_weights(d, seed)
+            Xc = synth.gmu_inputs(d, seed, rows=L, tag="X_cross")
+            run = lambda: ref.sambay_mlp_gmu_ref(Xc, X, mw["W_g"], mw["W_u"], gw["W1"], gw["W2"], residual=True)
+            what = "SwiGLU memory + GMU layer"
+        while reps < reps_max and (reps == 0 or time.perf_counter() - t0 < budget_s):
+            run()
+            reps += 1
+        el = time.perf_counter() - t0
+        return {"value": reps * L / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"the first {L} tokens ({what}) x {reps}, {el:.1f} s of float64 NumPy"}
     w = synth.scan_weights(d, seed)
     gws = [synth.gmu_weights(d, seed, layer=l) for l in range(layers)]
     if decode:
@@ -364,7 +402,8 @@ def prefill_kernel_work(name, d, layers, sms, peaks, peak_kind):
         peak = SFU_EX2_PER_SM_CLK * sms * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e9
         return "alu", T * Di * N, "Gexp/s", peak, \
             f"SFU ex2: {SFU_EX2_PER_SM_CLK}/SM/clk x {sms} SMs x max SM clock ({peak_kind} clock)"
-    if name in ("gmu_gate_gemm", "gmu_gate_gemm+tail", "gmu_out_gemm", "gmu_out_gemm+tail"):
+    if name in ("gmu_gate_gemm", "gmu_gate_gemm+tail", "gmu_out_gemm", "gmu_out_gemm+tail",
+                "in_proj", "in_proj+tail", "mlp_up", "mlp_up+tail", "mlp_gate", "mlp_gate+tail"):
         return "tensor", 2.0 * T * Dm * Di, "TFLOP/s", peaks["bf16_tflops"], f"{peak_kind} burst bf16"
     if name == "conv_silu":      # u in (bf16), uc split pair out (2 x bf16)
         return "hbm", T * Di * (2 + 4), "GB/s", hbm, f"{peak_kind} HBM copy"
@@ -377,11 +416,39 @@ def prefill_kernel_work(name, d, layers, sms, peaks, peak_kind):
     return None
 
 
+def kernel_report(name, per_kernel, kt_steps, d, layers, sms, peaks, peak_kind):
+    """Per-kernel entries (time, algorithmic work, achieved rate against the
+    peak) of a prefill-shaped step, and the roofline of the dominant one."""
+    kernels = []
+    for kname, ms_list in per_kernel.items():
+        cnt = len(ms_list) / kt_steps
+        ms = statistics.mean(ms_list)
+        entry = {"kernel": kname, "launches_per_step": cnt, "ms": ms}
+        kw = prefill_kernel_work(kname, d, layers, sms, peaks, peak_kind)
+        if kw is not None:
+            bound, units, unit, peak, note = kw
+            scale = 1e12 if unit == "TFLOP/s" else 1e9
+            achieved = units / (ms / 1e3) / scale
+            entry.update({"bound": bound, "algorithmic_per_launch": units, "achieved": achieved,
+                          "peak": peak, "unit": unit, "frac": achieved / peak, "peak_note": note})
+        kernels.append(entry)
+    kernels.sort(key=lambda e: -e["ms"] * e["launches_per_step"])
+    dom = kernels[0]
+    roofline = {"bound": dom.get("bound"), "achieved": dom.get("achieved"), "peak": dom.get("peak"),
+                "unit": dom.get("unit"), "frac": dom.get("frac"),
+                "traffic": DRAM_TRAFFIC_EARLIER_CAPTURE.get(dom["kernel"]) if name == HEADLINE else None,
+                "traffic_note": "from an earlier ncu capture of this kernel on this workload (unchanged "
+                                "kernel), else null",
+                "kernel": dom["kernel"], "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
+    return kernels, roofline
+
+
 def merge_tails(per_kernel):
     """A GEMM's K-split tail reduce finishes that GEMM: fold its time into the
     GEMM's entry (reported as '<gemm>+tail')."""
     out = dict(per_kernel)
-    for gemm, tail in (("gmu_out_gemm", "gmu_out_tail"), ("gmu_gate_gemm", "gmu_gate_tail")):
+    for gemm, tail in (("gmu_out_gemm", "gmu_out_tail"), ("gmu_gate_gemm", "gmu_gate_tail"),
+                       ("in_proj", "in_proj_tail"), ("mlp_up", "mlp_up_tail"), ("mlp_gate", "mlp_gate_tail")):
         if gemm in out and tail in out:
             a, b = out.pop(gemm), out.pop(tail)
             n = min(len(a), len(b))
@@ -527,27 +594,7 @@ def bench_prefill(args, ctx, name):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     assert abi.sambay_device_status() == 0
 
-    kernels = []
-    for kname, ms_list in per_kernel.items():
-        cnt = len(ms_list) / kt_steps
-        ms = statistics.mean(ms_list)
-        entry = {"kernel": kname, "launches_per_step": cnt, "ms": ms}
-        kw = prefill_kernel_work(kname, d, layers, sms, peaks, peak_kind)
-        if kw is not None:
-            bound, units, unit, peak, note = kw
-            scale = 1e12 if unit == "TFLOP/s" else 1e9
-            achieved = units / (ms / 1e3) / scale
-            entry.update({"bound": bound, "algorithmic_per_launch": units, "achieved": achieved,
-                          "peak": peak, "unit": unit, "frac": achieved / peak, "peak_note": note})
-        kernels.append(entry)
-    kernels.sort(key=lambda e: -e["ms"] * e["launches_per_step"])
-    dom = kernels[0]
-    roofline = {"bound": dom.get("bound"), "achieved": dom.get("achieved"), "peak": dom.get("peak"),
-                "unit": dom.get("unit"), "frac": dom.get("frac"),
-                "traffic": DRAM_TRAFFIC_EARLIER_CAPTURE.get(dom["kernel"]) if name == HEADLINE else None,
-                "traffic_note": "from an earlier ncu capture of this kernel on this workload (unchanged "
-                                "kernel), else null",
-                "kernel": dom["kernel"], "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
+    kernels, roofline = kernel_report(name, per_kernel, kt_steps, d, layers, sms, peaks, peak_kind)
     h2d = u.numel() * 2 + X0.numel() * 2
     return {
         "metric": METRICS[name], "value": value, "unit": UNIT, "ms_per_step": total_ms / steps,
@@ -559,6 +606,98 @@ def bench_prefill(args, ctx, name):
                 "d2h_bytes_per_step": sets[0]["out"].numel() * 2,
                 "note": "pinned host buffers; each step's copy-in and copy-out overlap its neighbours' compute "
                         "(two device buffer sets, separate copy streams)"},
+        "gpu_launches": launches * steps,
+    }
+
+
+# --------------------------------------------------------------------- our arm: f1 / f3 layers
+
+def bench_layer(args, ctx, name):
+    """The layers around the path at the headline sizes (batch 1, 2048 tokens,
+    d_model 2560, d_inner = d_ff 5120): the whole Mamba layer from X, or the
+    SambaY-MLP memory read by one GMU layer.  Same timing rules as the
+    headline (L2 flushed between steps, CUDA events on the stream)."""
+    import torch
+    from gated_memory_sharing_b200 import abi
+    from gated_memory_sharing_b200.layers import GMULayer, MambaLayer, MLPMemory
+    world, rank, device, flush, stream, peaks, peak_kind, sms = ctx
+    d, seed, layers, _ = workload_dims(name)
+    T, Dm, Di = d.tokens, d.d_model, d.d_inner
+    X = dev_normal((d.batch, d.seqlen, Dm), seed + 7919 * rank + 3, device)
+    if name == "mamba_layer_b1_l2048":
+        layer = MambaLayer(synth.scan_weights(d, seed), synth.mamba_block_weights(d, seed), Dm, abi.BF16)
+        h, cs = layer.scan.new_state(d.batch)
+        ins, out = [X], None
+
+        def step():
+            nonlocal out
+            out = layer.prefill(X, h, cs, fresh=True)[0]
+    else:
+        mw, gw = synth.mlp_weights(d, seed), synth.gmu_weights(d, seed)
+        mlp, gmu = MLPMemory(mw["W_g"], mw["W_u"], abi.BF16), GMULayer(gw["W1"], gw["W2"], abi.BF16)
+        X_self, X_cross = X.view(T, Dm), dev_normal((T, Dm), seed + 7919 * rank + 4, device)
+        M = torch.empty(T, Di, dtype=torch.bfloat16, device=device)
+        Y = torch.empty_like(X_cross)
+        ins, out = [X_self, X_cross], Y
+
+        def step():
+            mlp.forward(X_self, M)
+            gmu.forward(X_cross, M, residual=True, Y=Y)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert abi.sambay_device_status() == 0
+    steps = max(3, min(args.steps, 10))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush(i)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    value = world * steps * T / (total_ms / 1e3)
+
+    per_kernel, launches, kt_steps = {}, None, 3
+    for i in range(kt_steps):
+        flush(i)
+        with abi.KernelTimer(max_launches=64) as kt:
+            step()
+        torch.cuda.synchronize()
+        launches = len(kt.names)
+        for kname, ms in kt.durations_ms():
+            per_kernel.setdefault(kname, []).append(ms)
+    kernels, roofline = kernel_report(name, merge_tails(per_kernel), kt_steps, d, layers, sms, peaks, peak_kind)
+
+    # end to end: the inputs in from pinned host memory, the output back, per step
+    hosts = [t.cpu().pin_memory() for t in ins]
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        for t, hst in zip(ins, hosts):
+            t.copy_(hst, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    assert abi.sambay_device_status() == 0
+    return {
+        "metric": METRICS[name], "value": value, "unit": UNIT, "ms_per_step": total_ms / steps,
+        "steps": steps, "config": config_of(name, d, layers, False),
+        "l2": "flushed between steps (256 MB write, then a 256 MB read of another buffer so no dirty lines "
+              "remain; outside the step events)",
+        "roofline": roofline, "kernels": kernels,
+        "e2e": {"value": world * steps * T / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * 2 for t in ins), "d2h_bytes_per_step": out.numel() * 2},
         "gpu_launches": launches * steps,
     }
 
@@ -894,6 +1033,9 @@ def run_ours(args, world, rank, local):
             continue
         if name == "sambay2_prefill_b1_l2048":
             results[name] = bench_ssd(args, ctx, name)
+            continue
+        if name in LAYER_WORKLOADS:
+            results[name] = bench_layer(args, ctx, name)
             continue
         fn = bench_decode if workload_dims(name)[3] else bench_prefill
         results[name] = fn(args, ctx, name)
