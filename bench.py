@@ -392,8 +392,8 @@ def run_reference(args, world, rank):
 def prefill_kernel_work(name, d, layers, sms, peaks, peak_kind):
     """(bound, algorithmic units per launch, unit, peak, note) of one kernel of a
     prefill step.  Algorithmic = what the method must compute or move once:
-    exps for the scan, 2*M*N*K flops for a GMU GEMM (the out GEMM's K-split
-    tail reduction counts as part of the out GEMM), bytes read + written by the
+    exps for the scan, 2*M*N*K flops for a projection GEMM (its K-split tail,
+    summed inside the same kernel, included), bytes read + written by the
     memory-bound kernels (inputs once, outputs once)."""
     T, Di, Dm, N, R = d.tokens, d.d_inner, d.d_model, d.d_state, d.dt_rank
     ldx, Rp = R + 2 * N, (R + 63) // 64 * 64
@@ -402,8 +402,7 @@ def prefill_kernel_work(name, d, layers, sms, peaks, peak_kind):
         peak = SFU_EX2_PER_SM_CLK * sms * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e9
         return "alu", T * Di * N, "Gexp/s", peak, \
             f"SFU ex2: {SFU_EX2_PER_SM_CLK}/SM/clk x {sms} SMs x max SM clock ({peak_kind} clock)"
-    if name in ("gmu_gate_gemm", "gmu_gate_gemm+tail", "gmu_out_gemm", "gmu_out_gemm+tail",
-                "in_proj", "in_proj+tail", "mlp_up", "mlp_up+tail", "mlp_gate", "mlp_gate+tail"):
+    if name in ("gmu_gate_gemm", "gmu_out_gemm", "in_proj", "mlp_up", "mlp_gate"):
         return "tensor", 2.0 * T * Dm * Di, "TFLOP/s", peaks["bf16_tflops"], f"{peak_kind} burst bf16"
     if name == "conv_silu":      # u in (bf16), uc split pair out (2 x bf16)
         return "hbm", T * Di * (2 + 4), "GB/s", hbm, f"{peak_kind} HBM copy"
@@ -441,19 +440,6 @@ def kernel_report(name, per_kernel, kt_steps, d, layers, sms, peaks, peak_kind):
                                 "kernel), else null",
                 "kernel": dom["kernel"], "ms_per_launch": dom["ms"], "peak_note": dom.get("peak_note")}
     return kernels, roofline
-
-
-def merge_tails(per_kernel):
-    """A GEMM's K-split tail reduce finishes that GEMM: fold its time into the
-    GEMM's entry (reported as '<gemm>+tail')."""
-    out = dict(per_kernel)
-    for gemm, tail in (("gmu_out_gemm", "gmu_out_tail"), ("gmu_gate_gemm", "gmu_gate_tail"),
-                       ("in_proj", "in_proj_tail"), ("mlp_up", "mlp_up_tail"), ("mlp_gate", "mlp_gate_tail")):
-        if gemm in out and tail in out:
-            a, b = out.pop(gemm), out.pop(tail)
-            n = min(len(a), len(b))
-            out[gemm + "+tail"] = [a[i] + b[i] for i in range(n)]
-    return out
 
 
 def decode_bytes(d, B, layers):
@@ -537,7 +523,6 @@ def bench_prefill(args, ctx, name):
         launches = len(kt.names)
         for kname, ms in kt.durations_ms():
             per_kernel.setdefault(kname, []).append(ms)
-    per_kernel = merge_tails(per_kernel)
 
     # ---- end to end through the ABI with host buffers: every step copies its
     # inputs in from pinned host memory and its result out, as a serving loop
@@ -671,7 +656,7 @@ def bench_layer(args, ctx, name):
         launches = len(kt.names)
         for kname, ms in kt.durations_ms():
             per_kernel.setdefault(kname, []).append(ms)
-    kernels, roofline = kernel_report(name, merge_tails(per_kernel), kt_steps, d, layers, sms, peaks, peak_kind)
+    kernels, roofline = kernel_report(name, per_kernel, kt_steps, d, layers, sms, peaks, peak_kind)
 
     # end to end: the inputs in from pinned host memory, the output back, per step
     hosts = [t.cpu().pin_memory() for t in ins]

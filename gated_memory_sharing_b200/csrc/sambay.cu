@@ -7,10 +7,13 @@
 
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <vector>
+
+#include <unistd.h>
 
 #include "../../include/sambay.h"
 #include "common.cuh"
@@ -266,8 +269,30 @@ struct GmuWs {
 constexpr int kStepMaxRows = 256;
 constexpr int kStepMaxSplits = 8;
 // Partial tiles of a prefill GEMM's K-split tail: at most one 256 x 256 fp32
-// tile per CTA pair of a 148-SM B200.
+// tile per CTA pair of a 148-SM B200, then the tail units' arrival flags (one
+// 8-byte flag per tail unit and CTA of its pair) in an area of their own.
 constexpr int kTailUnits = 74;
+constexpr size_t kTailSyncBytes = 4096;
+
+// Epochs of the K-split tail's arrival flags: one per launch, from a 48-bit
+// sequence that starts at a point drawn from the clock and the process id
+// (splitmix64), so that no flag left in reused scratch carries a live epoch.
+unsigned long long next_tail_epoch() {
+  static const unsigned long long base = [] {
+    unsigned long long z = static_cast<unsigned long long>(
+                               std::chrono::steady_clock::now().time_since_epoch().count()) ^
+                           (static_cast<unsigned long long>(getpid()) << 32);
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }();
+  static std::atomic<unsigned long long> seq{0};
+  for (;;) {
+    const unsigned long long e = (base + seq.fetch_add(1)) & ((1ull << 48) - 1);
+    if (e != 0) return e;
+  }
+}
 
 GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
   GmuWs w{};
@@ -277,7 +302,7 @@ GmuWs gmu_ws_layout(const sambay_dims* d, long long rows, bool step) {
   if (!step && d->io == SAMBAY_BF16 && rows > 256) {
     // more than one 256-row tile: room for the K-split tail of either GEMM
     w.tail = off;
-    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4;
+    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4 + kTailSyncBytes;
     off += round256(w.tail_bytes);
   }
   w.total = off;
@@ -414,8 +439,8 @@ TailPlan tail_plan(int tiles, int BN, int slots, int min_width) {
 
 // K-split tail (pairs only): the partial wave's `ntail` tiles are each cut
 // along K into `splits` units of `kbps` k-blocks (ntail * splits <= slots);
-// every unit writes an fp32 partial tile and tail_reduce_kernel sums them in
-// split order and applies the epilogue.
+// every unit writes an fp32 partial tile; the GEMM's CTAs sum them in a fixed
+// order after their last unit and apply the epilogue.
 struct KTailPlan {
   int ntail = 0, splits = 1, kbps = 0;
 };
@@ -466,13 +491,13 @@ bool cluster_fits(int dev, int sms, int s, int count) {
 // `balance_tail` (no K split) applies
 // tail_plan, or for pairs with `tail_part` scratch of `tail_bytes` the
 // K-split tail when that leaves the shorter last round (a tail unit costs
-// 1/splits of a tile plus about a tenth of one for its partial tile and the
-// reduction, launched as `tail_name`).  PAIR: 256-row tiles on CTA pairs
-// (clusters of two).
+// 1/splits of a tile plus about a tenth of one for its partial tile and its
+// share of the reduction, which the same kernel's CTAs do after their last
+// unit).  PAIR: 256-row tiles on CTA pairs (clusters of two).
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW = 4, bool PAIR = false>
 sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
                      sambay::tc::GemmArgs g, int splits, cudaStream_t st, bool chained, bool balance_tail = false,
-                     float* tail_part = nullptr, size_t tail_bytes = 0, const char* tail_name = nullptr) {
+                     float* tail_part = nullptr, size_t tail_bytes = 0) {
   using namespace sambay::tc;
   using C = Cfg<BN, A_MN, B_MN, KIND, TRANS, EW, PAIR>;
   static bool attr_set[kMaxDevices] = {};
@@ -550,21 +575,25 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
   CUtensorMap tb2 = tb;
   g.tail_ksplit = 1;
   const int slots = PAIR ? pair_slots[dev] : sms;   // work units in flight at once
-  int ktail = 0;
   if (balance_tail && g.splits == 1) {
     // narrowest unit: 64 columns per CTA's B load (MN-major B: whole 64-column boxes)
     const int min_width = (PAIR && B_MN) ? 128 : 64;
     const TailPlan tp = tail_plan(g.tiles, BN, slots, min_width);
-    const KTailPlan kp = PAIR && tail_part ? ktail_plan(g.tiles, slots, g.k_blocks) : KTailPlan{};
+    // (the kernel sums a K-split tail only in its bf16 gate / residual epilogues)
+    constexpr bool kTailKind = KIND == sambay::tc::EPI_GATE || KIND == sambay::tc::EPI_RESID;
+    const KTailPlan kp = PAIR && kTailKind && tail_part ? ktail_plan(g.tiles, slots, g.k_blocks) : KTailPlan{};
     const double ncost = 1.0 / tp.nsplit, kcost = 1.0 / kp.splits + 0.1;
     if (kp.ntail > 0 && kcost < ncost &&
-        static_cast<size_t>(kp.ntail) * kp.splits * C::kBMT * BN * 4 <= tail_bytes) {
+        static_cast<size_t>(kp.ntail) * kp.splits * C::kBMT * BN * 4 + kTailSyncBytes <= tail_bytes &&
+        static_cast<size_t>(kp.ntail) * kp.splits * 2 * sizeof(unsigned long long) <= kTailSyncBytes) {
       g.full_tiles = g.tiles - kp.ntail;
       g.tail_ksplit = kp.splits;
       g.tail_kbps = kp.kbps;
       g.tail_part = tail_part;
+      g.tail_flags = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(tail_part) + tail_bytes -
+                                                           kTailSyncBytes);
+      g.tail_epoch = next_tail_epoch();
       g.tiles = g.full_tiles + kp.ntail * kp.splits;
-      ktail = kp.ntail;
     } else if (tp.nsplit > 1) {
       const int hb = (BN / tp.nsplit) / (PAIR ? 2 : 1);
       if (!B_MN && !make_map(&tb2, b.ptr, b.cols, b.rows, b.cols * 2, hb)) return SAMBAY_ERR_CUDA;
@@ -582,24 +611,6 @@ sambay_status run_tc(const char* name, int dev, int sms, Operand a, Operand b,
     const int cluster = PAIR ? 2 : g.csplit ? g.splits : 1;
     if (launch_k(kern, dim3(grid), dim3(gemm_threads(EW)), C::kSmem, st, chained, cluster, ta, tb, tb2, taux,
                  tout, g) != cudaSuccess)
-      return SAMBAY_ERR_CUDA;
-  }
-  if constexpr (PAIR) if (ktail > 0) {
-    if (cudaGetLastError() != cudaSuccess) return SAMBAY_ERR_CUDA;
-    const long long work = static_cast<long long>(ktail) * C::kBMT * (BN / 4) * kTailLanes;
-    auto rk = tail_reduce_kernel<BN, C::kBMT, KIND>;
-    SAMBAY_MAX_CARVEOUT(rk, dev);
-    // one resident wave (the grid-stride loop takes the rest): a second wave
-    // would pay the partials' L2 round trip again
-    static int per_sm[kMaxDevices] = {};
-    if (per_sm[dev] == 0) {
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rk, 256, 0) != cudaSuccess || n < 1) n = 1;
-      per_sm[dev] = n;
-    }
-    const int grid = static_cast<int>(std::min<long long>((work + 255) / 256, static_cast<long long>(per_sm[dev]) * sms));
-    ProfScope ps(tail_name ? tail_name : "gemm_tail_reduce", st);
-    if (launch_k(rk, dim3(grid), dim3(256), 0, st, true, 1, g, ktail) != cudaSuccess)
       return SAMBAY_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? SAMBAY_OK : SAMBAY_ERR_CUDA;
@@ -1029,7 +1040,7 @@ sambay_status gmu_common_checks(const sambay_dims* d, int64_t rows, const void* 
 template <int KIND>
 sambay_status project_tc(int dev, int sms, long long rows, int N, int K, const void* X, const void* W,
                          const void* aux, void* Y, float* tail, size_t tail_bytes, const char* name,
-                         const char* tail_name, cudaStream_t st) {
+                         cudaStream_t st) {
   if (rows <= kStepMaxRows) {
     auto g = tc_args(N, static_cast<int>(rows), K, Y, N, aux);
     g.csplit = 1;
@@ -1042,7 +1053,7 @@ sambay_status project_tc(int dev, int sms, long long rows, int N, int K, const v
   }
   return run_tc<256, false, false, KIND, false, 8, true>(name, dev, sms, Operand{X, rows, K}, Operand{W, N, K},
                                                          tc_args(static_cast<int>(rows), N, K, Y, N, aux), 1, st,
-                                                         false, true, tail, tail_bytes, tail_name);
+                                                         false, true, tail, tail_bytes);
 }
 
 // Workspace of the projections: the K-split tail's partial tiles (more than
@@ -1058,7 +1069,7 @@ ProjWs proj_ws_layout(const sambay_dims* d, long long rows, bool buffer) {
   if (buffer) off += round256(static_cast<size_t>(rows) * d->d_inner * io_bytes(d->io));
   if (d->io == SAMBAY_BF16 && rows > kStepMaxRows) {
     w.tail = off;
-    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4;
+    w.tail_bytes = static_cast<size_t>(kTailUnits) * 256 * 256 * 4 + kTailSyncBytes;
     off += round256(w.tail_bytes);
   }
   w.total = off;
@@ -1258,11 +1269,11 @@ sambay_status gmu_forward(const sambay_dims* d, int64_t rows, const void* X, con
   // G = X W1^T, epilogue H = M ⊙ SiLU(G)
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 4, true>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, false,
-      true, tail, L.tail_bytes, "gmu_gate_tail")));
+      true, tail, L.tail_bytes)));
   // Y = H W2 (+ residual); W2 [Di, Dm] is the MN-major B operand
   SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_RESID, false, 4, true>(
       "gmu_out_gemm", dev, sms, Operand{H, rows, Di}, Operand{W2, Di, Dm}, tc_args(T, Dm, Di, Y, Dm, residual), 1,
-      st, true, true, tail, L.tail_bytes, "gmu_out_tail")));
+      st, true, true, tail, L.tail_bytes)));
   return SAMBAY_OK;
 }
 
@@ -1283,7 +1294,7 @@ sambay_status gmu_forward_partial(const sambay_dims* d, int64_t rows, const void
   float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
   SAMBAY_TRY((run_tc<256, false, false, sambay::tc::EPI_GATE, false, 4, true>(
       "gmu_gate_gemm", dev, sms, Operand{X, rows, Dm}, Operand{W1, Di, Dm}, tc_args(T, Di, Dm, H, Di, M), 1, st, false,
-      true, tail, L.tail_bytes, "gmu_gate_tail")));
+      true, tail, L.tail_bytes)));
   // Y_part = H W2 in fp32: single-CTA 128 x 256 tiles (the CTA-pair form has
   // only the bf16 epilogues), whole tiles only
   SAMBAY_TRY((run_tc<256, false, true, sambay::tc::EPI_F32_PARTIAL, false, 4>(
@@ -1427,7 +1438,7 @@ sambay_status sambay_in_proj(const sambay_dims* d, int64_t rows, const void* X, 
                   static_cast<int>(rows), Di, Dm, static_cast<float*>(u), Di), st);
   float* tail = L.tail_bytes ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.tail) : nullptr;
   return project_tc<sambay::tc::EPI_RESID>(dev, sms, rows, Di, Dm, X, W_in, nullptr, u, tail, L.tail_bytes,
-                                           "in_proj", "in_proj_tail", st);
+                                           "in_proj", st);
 }
 
 size_t sambay_mlp_memory_workspace(const sambay_dims* d, int64_t rows) {
@@ -1460,9 +1471,9 @@ sambay_status sambay_mlp_memory(const sambay_dims* d, int64_t rows, const void* 
   float* tail = L.tail_bytes ? reinterpret_cast<float*>(w8 + L.tail) : nullptr;
   // U = X W_u^T, then M = U ⊙ SiLU(X W_g^T): the gate GEMM with U as its aux
   SAMBAY_TRY(project_tc<sambay::tc::EPI_RESID>(dev, sms, rows, Df, Dm, X, W_u, nullptr, U, tail, L.tail_bytes,
-                                               "mlp_up", "mlp_up_tail", st));
+                                               "mlp_up", st));
   return project_tc<sambay::tc::EPI_GATE>(dev, sms, rows, Df, Dm, X, W_g, U, M, tail, L.tail_bytes, "mlp_gate",
-                                          "mlp_gate_tail", st);
+                                          st);
 }
 
 }  // extern "C"

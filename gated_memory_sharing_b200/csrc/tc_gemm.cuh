@@ -335,8 +335,12 @@ struct GemmArgs {
                       // partial wave of tiles spreads over more SMs; no K split)
   int tail_ksplit;    // > 1 instead: every tile after full_tiles is cut along K into
   int tail_kbps;      // tail_ksplit units of tail_kbps k-blocks, each writing its fp32
-  float* tail_part;   // partial tile [tail tile][split][tile rows][BN] to tail_part;
-                      // tail_reduce_kernel sums them and applies the epilogue
+  float* tail_part;   // partial tile [tail tile][split][tile rows][BN] to tail_part.
+                      // The tail units run first (at most one per CTA pair); before
+                      // its first whole tile's epilogue every CTA sums a share of
+                      // the tail outputs
+  unsigned long long* tail_flags;  // per tail unit and pair rank: the epoch once stored
+  unsigned long long tail_epoch;   // this launch's 48-bit epoch (never 0)
   int a_early;        // launched with programmatic dependent launch: the A operand does
                       // not depend on the kernel before this one, so the producer loads
                       // the first pipeline stages' A tiles before griddepcontrol.wait
@@ -545,6 +549,13 @@ template <int BN>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   TileCoord c;
   c.tailk = -1;
+  if (g.tail_ksplit > 1) {
+    // K-split tail units come first in the schedule: unit t < nt is tail unit
+    // t, the rest are the whole tiles.  With nt <= the number of CTA pairs,
+    // each pair meets at most one tail unit, before any whole tile.
+    const int nt = g.tiles - g.full_tiles;
+    t = t < nt ? g.full_tiles + t : t - nt;
+  }
   if (g.tail_ksplit > 1 && t >= g.full_tiles) {
     const int r = t - g.full_tiles;
     c.tailk = r / g.tail_ksplit;
@@ -586,6 +597,134 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& g, int t) {
   c.n0 = c.n * BN;
   c.bn = BN;
   return c;
+}
+
+// ---------------------------------------------------------------- K-split tail
+//
+// Each CTA of a tail unit, once its rows of the partial tile are stored,
+// writes this launch's epoch to its own flag in the caller's scratch (no
+// atomics: the arrivals of one launch land at the same moment and must not
+// queue on one word).  The flags' contents on entry are undefined; epochs come
+// from a 48-bit sequence that a process starts at a random point and never
+// repeats, so a flag holds the live epoch only once this launch has set it.
+
+constexpr int kMaxTailSplits = 16;
+constexpr int kTailLanes = 4;      // lanes summing one output's partials
+
+__device__ __forceinline__ void tail_flag_set(unsigned long long* f, unsigned long long epoch) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(epoch) : "memory");
+}
+
+// One warp: bounded wait until all n flags hold the epoch.  False (the same
+// in every lane) if the limit ran out (status recorded) or the CTA is aborting.
+__device__ __forceinline__ bool tail_flags_wait(const unsigned long long* f, int n, unsigned long long epoch,
+                                                volatile int* abort_flag, unsigned long long limit) {
+  const int lane = threadIdx.x & 31;
+  const long long t0 = clock64();
+  for (;;) {
+    bool mine = true;
+    for (int i = lane; i < n; i += 32) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f + i) : "memory");
+      mine &= v == epoch;
+    }
+    if (__all_sync(0xffffffffu, mine)) return true;
+    const bool late = static_cast<unsigned long long>(clock64() - t0) > limit;
+    if (__any_sync(0xffffffffu, *abort_flag != 0 || late)) {
+      if (lane == 0 && !*abort_flag) {
+        *abort_flag = 1;
+        record_status(kStatusTimeout);
+      }
+      return false;
+    }
+    __nanosleep(128);
+  }
+}
+
+// Sums the tail tiles' partials and applies the epilogue: output float4 groups
+// of kTailLanes lanes, warp w of `warps` taking groups w, w + warps, ...  The
+// lanes of a group sum every kTailLanes-th split, then combine by shuffles (a
+// fixed order: the result does not depend on which warp runs it).  A few
+// warps per SM run this, so each lane keeps the loads of kTailBatch groups in
+// flight at once.
+constexpr int kTailBatch = 4;
+
+template <int BN, int BMT, int KIND>
+__device__ __forceinline__ void tail_reduce_warps(const GemmArgs& g, int ntail, long long w0, long long warps) {
+  constexpr int Q = BN / 4, LPG = kTailLanes, PER = kMaxTailSplits / LPG, U = kTailBatch;
+  constexpr bool kAuxKind = KIND == EPI_GATE || KIND == EPI_RESID;
+  const int lane = threadIdx.x & 31, sub = lane % LPG;
+  const long long total = static_cast<long long>(ntail) * BMT * Q;   // output float4s
+  for (long long wb = w0; wb * (32 / LPG) < total; wb += U * warps) {
+    float4 x[U][PER];
+    uint2 aux4[U];
+    long long o[U];
+    int n[U];
+    bool live[U], vec4[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long e = (wb + u * warps) * (32 / LPG) + lane / LPG;
+      const int i = static_cast<int>(e / (BMT * Q));
+      const int lr = static_cast<int>((e / Q) % BMT), lq = static_cast<int>(e % Q);
+      const int tile = g.full_tiles + i;
+      const int m = (tile % g.m_tiles) * BMT + lr;
+      n[u] = (tile / g.m_tiles) * BN + 4 * lq;
+      live[u] = e < total && m < g.M && n[u] < g.N;
+      const float* base = g.tail_part + (static_cast<long long>(i) * g.tail_ksplit * BMT + lr) * BN + 4 * lq;
+      o[u] = static_cast<long long>(m) * g.ldo + n[u];
+      // the aux (M or the residual) of the reducing lane's 4 outputs, loaded
+      // together with the partials so the round trips overlap
+      vec4[u] = n[u] + 4 <= g.N && (o[u] & 3) == 0;
+      aux4[u] = make_uint2(0u, 0u);
+      if (kAuxKind && g.aux != nullptr && live[u] && sub == 0 && vec4[u])
+        aux4[u] = __ldcg(reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(g.aux) + o[u]));
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int sp = sub + j * LPG;
+        const bool on = live[u] && sp < g.tail_ksplit;
+        x[u][j] = ldcg_or_zero(base + (on ? static_cast<long long>(sp) * BMT * BN : 0), on);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float4 acc = x[u][0];
+#pragma unroll
+      for (int j = 1; j < PER; ++j) {
+        acc.x += x[u][j].x; acc.y += x[u][j].y; acc.z += x[u][j].z; acc.w += x[u][j].w;
+      }
+#pragma unroll
+      for (int off = LPG / 2; off >= 1; off >>= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+      }
+      if (!live[u] || sub != 0) continue;
+      const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+      if (kAuxKind && vec4[u]) {
+        // 4 bf16 outputs as one 8-byte store
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&aux4[u]);
+        const float2 a01 = __bfloat1622float2(a2[0]), a23 = __bfloat1622float2(a2[1]);
+        const float a[4] = {a01.x, a01.y, a23.x, a23.y};
+        float r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = KIND == EPI_GATE ? silu(v[j]) * a[j] : v[j] + a[j];
+        uint2 packed;
+        *reinterpret_cast<__nv_bfloat162*>(&packed.x) = __floats2bfloat162_rn(r[0], r[1]);
+        *reinterpret_cast<__nv_bfloat162*>(&packed.y) = __floats2bfloat162_rn(r[2], r[3]);
+        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(g.out) + o[u]) = packed;
+        continue;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (n[u] + j >= g.N) break;
+        float a = 0.0f;
+        if (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr))
+          a = to_f32(reinterpret_cast<const bf16*>(g.aux)[o[u] + j]);
+        epi_store_one<KIND>(g, o[u] + j, n[u] + j, v[j], a);
+      }
+    }
+  }
 }
 
 template <int BN, bool A_MN, bool B_MN, int KIND, bool TRANS, int EW, bool PAIR>
@@ -844,6 +983,9 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
     uint32_t acc_phase = 0;
     uint32_t aux_phase = 0;    // parity bit per aux slot
     int sp_local = 0;          // softplus chunks this warp has staged (slot double buffering)
+    bool tail_summed = false;  // this CTA's share of the K-split tail outputs is done
+    // the K-split tail: CTA pairs with a bf16 epilogue (the host plans it for no other)
+    constexpr bool kTailCode = PAIR && (KIND == EPI_GATE || KIND == EPI_RESID);
     const bool has_aux = KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr);
     for (int t = unit0; t < g.tiles; t += ustride) {
       const TileCoord c = tile_coord<BN>(g, t);
@@ -867,6 +1009,29 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
         if (KIND == EPI_SOFTPLUS)
           for (int i = ep_tid; i < c.bn; i += EPI_THREADS)
             epi_vec[i] = c.n0 + i < g.N ? g.vec[c.n0 + i] : 0.0f;
+      }
+      if constexpr (kTailCode) if (g.tail_ksplit > 1 && c.tailk < 0 && !tail_summed) {
+        // The CTA's first whole tile.  Every CTA pair ran its tail unit (if
+        // any) first, so the tail's partials are in or nearly so: once every
+        // flag is (both CTAs of every tail unit), this CTA's epilogue warps sum
+        // their share of the tail outputs while the tile's main loop runs on
+        // the tensor cores.  One warp waits; the barrier hands its verdict (an
+        // aborting CTA skips the sum) to the others.
+        tail_summed = true;
+        const int nt = g.tiles - g.full_tiles;
+        named_bar_sync<EPI_THREADS>();
+        if (warp == 2) {
+          const bool in = tail_flags_wait(g.tail_flags, 2 * nt, g.tail_epoch, abort_flag,
+                                          g.wait_limit ? g.wait_limit : kWaitCycles);
+          if (lane == 0) *last_flag = in ? 1 : 0;
+        }
+        named_bar_sync<EPI_THREADS>();
+        if (*last_flag) {
+          __threadfence();
+          tail_reduce_warps<BN, C::kBMT, KIND>(g, nt / g.tail_ksplit,
+                                               static_cast<long long>(blockIdx.x) * EW + (warp - 2),
+                                               static_cast<long long>(gridDim.x) * EW);
+        }
       }
       bool ok = true;
       // stall_test: auxf[3] is never armed in the element-wise (TRANS) epilogue,
@@ -1092,6 +1257,12 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
         }
         named_bar_sync<EPI_THREADS>();
       }
+      if constexpr (kTailCode) if (c.tailk >= 0) {
+        // this CTA's rows of a K-split tail unit are stored: publish them
+        __threadfence();
+        named_bar_sync<EPI_THREADS>();
+        if (ep_tid == 0) tail_flag_set(g.tail_flags + 2 * (c.tailk * g.tail_ksplit + c.split) + rank, g.tail_epoch);
+      }
     }
   }
 
@@ -1233,87 +1404,6 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                    "r"(C::kTmemCols)
                    : "memory");
-  }
-}
-
-// The K-split tail tiles of a GEMM: out = epilogue(sum of the tail_ksplit
-// (<= kMaxTailSplits) partial tiles).  kTailLanes lanes share one output
-// float4 (4 consecutive columns of a row): lane `sub` adds splits sub,
-// sub + kTailLanes, ... in order, then a fixed xor tree combines the lanes,
-// so the result is the same on every run.  Warps iterate uniformly (shuffles
-// need all lanes).
-constexpr int kMaxTailSplits = 16;
-constexpr int kTailLanes = 4;
-
-template <int BN, int BMT, int KIND>
-__global__ void __launch_bounds__(256) tail_reduce_kernel(const GemmArgs g, int ntail) {
-  pdl_wait();
-  pdl_launch_dependents();
-  constexpr int Q = BN / 4, LPG = kTailLanes, PER = kMaxTailSplits / LPG;
-  const int lane = threadIdx.x & 31, sub = lane % LPG;
-  const long long total = static_cast<long long>(ntail) * BMT * Q;   // output float4s
-  const long long warps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
-  for (long long w = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
-       w * (32 / LPG) < total; w += warps) {
-    const long long e = w * (32 / LPG) + lane / LPG;
-    const int i = static_cast<int>(e / (BMT * Q));
-    const int lr = static_cast<int>((e / Q) % BMT), lq = static_cast<int>(e % Q);
-    const int tile = g.full_tiles + i;
-    const int m = (tile % g.m_tiles) * BMT + lr;
-    const int n = (tile / g.m_tiles) * BN + 4 * lq;
-    const bool live = e < total && m < g.M && n < g.N;
-    const float* base = g.tail_part + (static_cast<long long>(i) * g.tail_ksplit * BMT + lr) * BN + 4 * lq;
-    const long long o = static_cast<long long>(m) * g.ldo + n;
-    // the aux (M or the residual) of the reducing lane's 4 outputs, loaded
-    // together with the partials so the two round trips overlap
-    constexpr bool kAuxKind = KIND == EPI_GATE || KIND == EPI_RESID;
-    const bool vec4 = n + 4 <= g.N && (o & 3) == 0;
-    uint2 aux4 = make_uint2(0u, 0u);
-    if (kAuxKind && g.aux != nullptr && live && sub == 0 && vec4)
-      aux4 = __ldcg(reinterpret_cast<const uint2*>(reinterpret_cast<const bf16*>(g.aux) + o));
-    float4 x[PER];
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int sp = sub + j * LPG;
-      const bool on = live && sp < g.tail_ksplit;
-      x[j] = ldcg_or_zero(base + (on ? static_cast<long long>(sp) * BMT * BN : 0), on);
-    }
-    float4 acc = x[0];
-#pragma unroll
-    for (int j = 1; j < PER; ++j) {
-      acc.x += x[j].x; acc.y += x[j].y; acc.z += x[j].z; acc.w += x[j].w;
-    }
-#pragma unroll
-    for (int off = LPG / 2; off >= 1; off >>= 1) {
-      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
-      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
-      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-    }
-    if (!live || sub != 0) continue;
-    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-    if (kAuxKind && vec4) {
-      // 4 bf16 outputs as one 8-byte store
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&aux4);
-      const float2 a01 = __bfloat1622float2(a2[0]), a23 = __bfloat1622float2(a2[1]);
-      const float a[4] = {a01.x, a01.y, a23.x, a23.y};
-      float r[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) r[j] = KIND == EPI_GATE ? silu(v[j]) * a[j] : v[j] + a[j];
-      uint2 packed;
-      *reinterpret_cast<__nv_bfloat162*>(&packed.x) = __floats2bfloat162_rn(r[0], r[1]);
-      *reinterpret_cast<__nv_bfloat162*>(&packed.y) = __floats2bfloat162_rn(r[2], r[3]);
-      *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(g.out) + o) = packed;
-      continue;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (n + j >= g.N) break;
-      float a = 0.0f;
-      if (KIND == EPI_GATE || (KIND == EPI_RESID && g.aux != nullptr))
-        a = to_f32(reinterpret_cast<const bf16*>(g.aux)[o + j]);
-      epi_store_one<KIND>(g, o + j, n + j, v[j], a);
-    }
   }
 }
 

@@ -211,8 +211,10 @@ SAMBAY_API sambay_status sambay_scan_step(const sambay_scan_weights* w, const sa
  * Two tensor-core GEMMs: G = X W1^T with SiLU(G) ⊙ M fused into its
  * epilogue (H, io, kept in ws), then H W2 with the residual fused.  In bf16
  * with more than 256 rows, ws also holds the fp32 partial tiles of a GEMM
- * whose last round of tiles is split along K (summed in a fixed order, so
- * results do not vary from run to run).
+ * whose last round of tiles is split along K, and flags marking their
+ * arrival; the same kernel sums them in a fixed order, so results do not
+ * vary from run to run.  ws needs no initialisation, but two calls in flight
+ * at once must not share it.
  */
 SAMBAY_API sambay_status gmu_forward(const sambay_dims* dims, int64_t rows, const void* X, const void* M,
                           const void* W1, const void* W2, const void* residual, void* Y,

@@ -155,8 +155,8 @@ def test_workspace_queries(lib):
     assert abi.sambay_scan_prefill_workspace(f) == r256(64 * 128 * 4) + r256(64 * 36 * 4) + r256(64 * 128 * 4) \
         + r256(32 * 64 * 4)
     # H, then (more than one 256-row tile) one fp32 256 x 256 partial tile per
-    # CTA pair of 148 SMs for a GEMM's K-split tail
-    assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2) + r256(74 * 256 * 256 * 4)
+    # CTA pair of 148 SMs for a GEMM's K-split tail, and their arrival flags
+    assert abi.gmu_forward_workspace(d, 2048) == r256(2048 * 5120 * 2) + r256(74 * 256 * 256 * 4 + 4096)
     assert abi.gmu_forward_workspace(d, 256) == r256(256 * 5120 * 2)
     # H only: the decode GEMMs reduce their K splits in shared memory
     assert abi.gmu_step_workspace(d, 64) == r256(64 * 5120 * 2)

@@ -81,7 +81,8 @@ def test_gmu_forward_multi_tile_bf16():
 ])
 def test_gmu_forward_k_split_tail_bf16(rows, d_model, d_inner):
     # more 256-row tiles than CTA pairs: the partial last round runs as K
-    # ranges whose fp32 partial tiles a second kernel sums in split order
+    # ranges (first, one per CTA pair) whose fp32 partial tiles the same
+    # kernel's CTAs sum in a fixed order after their last whole tile
     d = synth.Dims(1, 1, d_model, d_inner, 16, 4, 16, synth.BF16)
     seed = 15
     gw = synth.gmu_weights(d, seed)
@@ -91,7 +92,12 @@ def test_gmu_forward_k_split_tail_bf16(rows, d_model, d_inner):
     Y = g.forward(to_device(X, abi.BF16), to_device(M, abi.BF16), residual=True)
     Yr, _, _ = ref.gmu_ref(X, M, gw["W1"], gw["W2"], residual=True)
     assert_close(host(Y), Yr, TOL_BF16, f"gmu_forward K-split tail rows={rows}")
-    # deterministic: the same bits on a second call
+    # deterministic: the same bits on a second call, whatever the scratch holds
+    # on entry (the tail's arrival word included: random bytes here)
+    ws = g._ws[("fwd", rows)]
+    gen = torch.Generator(device=ws.device)
+    gen.manual_seed(rows)
+    ws.copy_(torch.randint(0, 256, ws.shape, generator=gen, device=ws.device, dtype=torch.int32).to(ws.dtype))
     assert torch.equal(Y, g.forward(to_device(X, abi.BF16), to_device(M, abi.BF16), residual=True))
 
 
