@@ -25,9 +25,10 @@
 // Tile 128 x BN x 64, SWIZZLE_128B smem layout (what TMA writes with a 128-byte
 // inner box), UMMA smem descriptors per the sm_100 matrix-descriptor format.
 //
-// Every mbarrier wait is bounded (clock64); on expiry the kernel records
-// SAMBAY_ERR_TIMEOUT in the device status word, raises a CTA-wide abort flag,
-// drains its in-flight TMA loads and MMAs (again bounded), frees TMEM and
+// Every mbarrier wait is bounded (clock64), and so is the wait for the K-split
+// tail's arrival flags (other CTAs' partial tiles); on expiry the kernel
+// records SAMBAY_ERR_TIMEOUT in the device status word, raises a CTA-wide abort
+// flag, drains its in-flight TMA loads and MMAs (again bounded), frees TMEM and
 // returns.
 #pragma once
 
