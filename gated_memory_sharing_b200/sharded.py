@@ -23,6 +23,8 @@ between GPUs).
 
 from __future__ import annotations
 
+import contextlib
+
 import numpy as np
 import torch
 
@@ -106,6 +108,11 @@ class DeviceOps:
         abi.gmu_finish(self.gmu.dims(rows), rows, Y_sum, residual, Y, stream)
 
 
+def _on(stream):
+    """Make `stream` torch's current stream for the block (no-op for None)."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _dist_all_reduce(t: torch.Tensor) -> None:
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
@@ -127,7 +134,8 @@ class ShardedPrefill:
                 stream=None):
         """u [B, L, Di_shard] (this rank's channels), X [B*L, d_model]
         (replicated) -> M [B, L, Di_shard], Y [B*L, d_model].  States are
-        this rank's channels, updated in place."""
+        this rank's channels, updated in place.  With `stream` given, the
+        all-reduces are issued on it too, between the calls they join."""
         B, L, _ = u.shape
         rows = B * L
         if fresh is None:
@@ -140,10 +148,12 @@ class ShardedPrefill:
             Y = torch.empty_like(X)
         xdbl = self.ops.xdbl_buffer(rows)
         self.ops.xproj(u, conv_state, fresh, xdbl, stream)
-        self.all_reduce(xdbl)                       # [delta | B | C] summed over all channels
+        with _on(stream):
+            self.all_reduce(xdbl)                   # [delta | B | C] summed over all channels
         self.ops.finish(u, xdbl, M, ssm_state, conv_state, fresh, stream)
         y_part = self.ops.y_buffer(rows)
         self.ops.gmu_partial(X, M.reshape(rows, -1), y_part, stream)
-        self.all_reduce(y_part)                     # H W2 summed over all channels
+        with _on(stream):
+            self.all_reduce(y_part)                 # H W2 summed over all channels
         self.ops.gmu_finish(y_part, X if residual else None, Y, stream)
         return M, Y, ssm_state, conv_state
