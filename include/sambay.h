@@ -263,7 +263,9 @@ SAMBAY_API sambay_status gmu_step(const sambay_dims* dims, int64_t rows, const v
  *
  *   X [rows, Dm] io;  W_in [Di, Dm] io (used transposed);  u [rows, Di] io out
  *   (must not alias X).  ws: >= sambay_in_proj_workspace(dims, rows) (the
- *   K-split tail partials of a bf16 GEMM of more than 256 rows; else 0).
+ *   K-split tail partials of a bf16 GEMM of more than 256 rows and their
+ *   arrival flags; else 0), no initialisation needed, not shared by two calls
+ *   in flight at once.
  * Up to 256 rows (decode) W_in streams once through the swap-AB decode GEMM.
  */
 SAMBAY_API size_t sambay_in_proj_workspace(const sambay_dims* dims, int64_t rows);
